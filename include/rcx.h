@@ -1,0 +1,220 @@
+/*
+ * rcx.h -- C ABI of librcx.so: context-extended attention forward on B200.
+ *
+ * The library computes the long-context attention forward pass described by
+ * the source pages: RoPE frequencies under a scaled schedule, rotation of Q
+ * and K, blockwise causal attention with an online softmax over KV blocks
+ * visited in Ring-Attention order, and the LSE merge of partial results.
+ *
+ * Conventions for every entry point:
+ *   - Plain pointers and sizes only.  Tensors are passed as rcx_tensor views:
+ *     a DEVICE pointer, a dtype, a 4-D shape and element strides.  Q, K, V and
+ *     O use [B, N, H, d] (batch, token, head, head_dim) with stride[3] == 1.
+ *     LSE tensors use [B, H, N, 1] (fp32, stride[3] ignored).
+ *   - The caller owns every buffer.  No entry point allocates device memory
+ *     except rcx_ring_attn_fwd_host, which stages its own device copies.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL means
+ *     the legacy default stream).  Argument errors are detected on the host
+ *     and returned before anything is launched.
+ *   - Errors are returned as rcx_status codes; nothing throws across the ABI.
+ *     A kernel whose bounded wait runs out records RCX_ERR_DEVICE_TIMEOUT in a
+ *     device status word that rcx_device_status() reads.
+ *   - Citations name the source page and the section that defines the step.
+ */
+#ifndef RCX_H
+#define RCX_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RCX_OK = 0,
+    RCX_ERR_INVALID_ARG = -1,    /* bad shape, stride, scheme or NULL pointer  */
+    RCX_ERR_UNSUPPORTED = -2,    /* valid request this build has no path for  */
+    RCX_ERR_ALIGNMENT = -3,      /* pointer or stride breaks a vector/TMA rule */
+    RCX_ERR_CUDA = -4,           /* a CUDA runtime/driver call failed          */
+    RCX_ERR_DEVICE_TIMEOUT = -5  /* a device-side bounded wait gave up         */
+} rcx_status;
+
+typedef enum { RCX_F32 = 0, RCX_BF16 = 1 } rcx_dtype;
+
+/* RoPE frequency schedules (see rcx_rope_freqs). */
+typedef enum {
+    RCX_ROPE_PLAIN = 0,      /* theta_i = base^(-2i/d)                              */
+    RCX_ROPE_PI = 1,         /* position interpolation m -> m/s                     */
+    RCX_ROPE_NTK = 2,        /* base' = base * s^(d/(d-2))                          */
+    RCX_ROPE_DYN_NTK = 3,    /* base'(l) with l = L_target, factor 1 if l <= L_train */
+    RCX_ROPE_NTK_PARTS = 4,  /* per-pair wavelength bands alpha/beta                 */
+    RCX_ROPE_YARN = 5        /* NTK-by-parts frequencies + temperature t            */
+} rcx_rope_scheme;
+
+/* Which operands an attention call rotates in-kernel (rope_flags). */
+enum { RCX_ROTATE_Q = 1, RCX_ROTATE_K = 2 };
+
+typedef struct {
+    void* ptr;           /* device pointer (host pointer for the *_host calls) */
+    int32_t dtype;       /* rcx_dtype                                           */
+    int64_t shape[4];
+    int64_t stride[4];   /* in elements                                         */
+} rcx_tensor;
+
+/* Version of the ABI (major * 100 + minor). */
+int rcx_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* rcx_status_string(int status);
+
+/*
+ * rcx_rope_freqs -- per-pair rotation frequencies theta'_i, i < d/2, and the
+ * attention temperature t, in float64 on the host.
+ *
+ *   theta_i = base^(-2i/d)              ("Context Extension" concept page,
+ *                                        RoPE scaling schemes / Technical principles)
+ *   s = L_target / L_train
+ *   PI:        theta_i / s              ("Context window extension: 4K to 1M" 2.1;
+ *                                        the page's m -> m/s, folded into theta)
+ *   NTK:       base' = base s^(d/(d-2)) (same page 2.2)
+ *   DYN_NTK:   base'(l), l = L_target; factor 1 when l <= L_train (same page 3)
+ *   NTK_PARTS: theta_i * f(lambda_i), lambda_i = 2 pi / theta_i; f = 1 below
+ *              L_train/beta, 1/s above L_train/alpha, linear in lambda between
+ *              (same page 2.3, band reading of the garbled code)
+ *   YARN:      NTK_PARTS frequencies and t = 0.1 ln s + 1 (same page 2.4)
+ * t = 1 for every scheme but YARN.
+ *
+ * d: even, 2..256.  L_train, L_target > 0.  alpha, beta used by NTK_PARTS and
+ * YARN only (0 < alpha < beta).  inv_freq_out: caller-owned host array of d/2
+ * doubles.  temperature_out: host double, may be NULL.
+ * Returns RCX_ERR_INVALID_ARG on a bad argument (outputs untouched).
+ */
+int rcx_rope_freqs(int scheme, double base, int d, int64_t L_train, int64_t L_target,
+                   double alpha, double beta, double* inv_freq_out, double* temperature_out);
+
+/*
+ * rcx_rope_apply -- rotate Q and/or K by R(m) ("Context Extension" concept page,
+ * Technical principles: each pair of dimensions (2i, 2i+1) turns by
+ * phi = m * theta'_i; q_m = R(m) W_q x_m, k_n = R(n) W_k x_n).
+ *
+ * q, k: [B, N, H, d] inputs (bf16 or f32); q_out, k_out: outputs of the same
+ * shape and dtype (out.ptr == in.ptr rotates in place; an operand whose
+ * in.ptr is NULL is skipped).  positions: device int64 array of n_positions
+ * >= N entries, position of token n is positions[n]; NULL means m = n.
+ * inv_freq: HOST array of d/2 doubles (from rcx_rope_freqs).
+ * Angles are reduced modulo 2 pi in float64 before an fp32 sincos, so the
+ * applied angle is within about 5e-7 rad of m * theta' for every m < 2^24.
+ * Memory-bound; data path: read x, write x' once.
+ */
+int rcx_rope_apply(rcx_tensor q, rcx_tensor k, rcx_tensor q_out, rcx_tensor k_out,
+                   const int64_t* positions, int64_t n_positions,
+                   const double* inv_freq, void* stream);
+
+/*
+ * rcx_attn_blockwise_fwd -- causal attention forward with an online softmax
+ * over KV tiles ("Context Extension" concept page, FlashAttention section:
+ * B_r x B_c tiles in on-chip memory, running max, O(n) memory), GQA
+ * (query head h reads KV head h / (Hq/Hkv)), optional sliding window of
+ * `window` keys with `n_sink` StreamingLLM sink keys ("Context window
+ * extension: 4K to 1M" 4.1 and 4.2), logits scaled by 1/(sqrt(d) t)
+ * (t from rcx_rope_freqs, same page 2.4).
+ *
+ * q: [B, Nq, Hq, d]; k, v: [B, Nk, Hkv, d]; o: [B, Nq, Hq, d] (bf16 or f32);
+ * lse: [B, Hq, Nq, 1] fp32 natural-log LSE of the scaled logits, ptr may be
+ * NULL.  Query row i is global token q_start + i, key j is k_start + j; the
+ * mask is  j <= i  and (window == 0 or i - window < j or j < n_sink).
+ * A row with no visible key gets O = 0 and lse = -inf.
+ *
+ * kv_block: Ring-Attention block size in keys (0 = the whole sequence is one
+ * block).  The KV tiles of a query tile in shard r = i / kv_block are visited
+ * in ring order, blocks (r - t) mod P for t = 0, 1, ... ("Context window
+ * extension: 4K to 1M" 5.3, kwkr.cn 2.2); the online softmax merges them.
+ * The result does not depend on kv_block beyond rounding.
+ *
+ * rope_flags: RCX_ROTATE_Q / RCX_ROTATE_K rotate that operand in-kernel with
+ * inv_freq (HOST, d/2 doubles) at positions[global token] (device int64,
+ * n_positions entries; NULL = identity).  rope_flags == 0: Q and K are taken
+ * as already rotated.
+ *
+ * Paths: f32 inputs run a SIMT fp32 kernel (any d <= 128, even).  bf16 inputs
+ * with d == 128 run the tcgen05/TMEM tensor-core kernel; it rotates Q in its
+ * tile load and needs K pre-rotated (RCX_ROTATE_K returns
+ * RCX_ERR_UNSUPPORTED there: rotate K once with rcx_rope_apply).
+ * Alignment: bf16 tensor-core path needs 16-byte aligned base pointers and
+ * token/head strides that are multiples of 8 elements.
+ */
+int rcx_attn_blockwise_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o,
+                           rcx_tensor lse, int64_t kv_block, int64_t window, int64_t n_sink,
+                           double temperature, int64_t q_start, int64_t k_start,
+                           const int64_t* positions, int64_t n_positions,
+                           const double* inv_freq, int rope_flags, void* stream);
+
+/*
+ * rcx_merge_partials -- LSE-weighted merge of two partial results over
+ * disjoint key sets: m = max(lse_a, lse_b), w = exp(lse - m),
+ * o = (w_a o_a + w_b o_b) / (w_a + w_b), lse = m + ln(w_a + w_b).
+ * This is the page's "output += block_output" of the Ring Attention loop
+ * ("Context window extension: 4K to 1M" 5.3) made exact, and the online
+ * aggregation of kwkr.cn 2.2.
+ *
+ * o_a, o_b: [B, N, H, d] fp32; lse_a, lse_b: [B, H, N, 1] fp32.
+ * o_out / lse_out: result (o_out f32 or bf16); o_out.ptr == NULL writes the
+ * result back into (o_a, lse_a).  Two -inf partials give o = 0, lse = -inf.
+ * Memory-bound.
+ */
+int rcx_merge_partials(rcx_tensor o_a, rcx_tensor lse_a, rcx_tensor o_b, rcx_tensor lse_b,
+                       rcx_tensor o_out, rcx_tensor lse_out, void* stream);
+
+/*
+ * rcx_ring_attn_fwd -- the Ring-Attention schedule on one device: the
+ * sequence is cut into P = ceil(N / kv_block) blocks; at step t every query
+ * shard r attends to KV block (r - t) mod P ("Context window extension: 4K to
+ * 1M" 5.3: send to rank + 1, receive from rank - 1; kwkr.cn 2.2: roll the
+ * chunks by one), blocks with no visible key are skipped, and each step's
+ * partial is merged into an fp32 accumulator with rcx_merge_partials' rule.
+ * The final O is written in o's dtype, lse (optional) as for the attention call.
+ *
+ * q, k, v, o, lse, window, n_sink, temperature, positions, inv_freq,
+ * rope_flags: as rcx_attn_blockwise_fwd (q_start = k_start = 0).  With
+ * RCX_ROTATE_K on the bf16 path, K is rotated once into the workspace.
+ * workspace: device buffer of at least rcx_ring_workspace_size() bytes,
+ * 256-byte aligned, owned by the caller.
+ */
+int64_t rcx_ring_workspace_size(rcx_tensor q, rcx_tensor k, int64_t kv_block, int rope_flags);
+int rcx_ring_attn_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                      int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+                      const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                      int rope_flags, void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * Host<->device convenience for callers without device memory management:
+ * same as rcx_ring_attn_fwd but q, k, v, o (and lse if non-NULL) are HOST
+ * buffers (pinned for full copy speed); the call allocates the device copies
+ * and workspace, copies in, computes, copies out and frees, synchronously on
+ * `stream`.  positions is a HOST array here.
+ */
+int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                           int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+                           const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                           int rope_flags, void* stream);
+
+/*
+ * Device status word: kernels with bounded waits record the first
+ * RCX_ERR_DEVICE_TIMEOUT here instead of hanging.  rcx_device_status()
+ * synchronises `stream`, stores the word in *status_out and clears it.
+ */
+int rcx_device_status(void* stream, int* status_out);
+
+/*
+ * Test hook: make the next tensor-core attention launches wait on a barrier
+ * that nothing arrives at, for `spins` iterations, so that the bounded-wait
+ * path is exercised (the kernel records RCX_ERR_DEVICE_TIMEOUT and returns).
+ * 0 switches it off.  Host-selected; no fault or trap is involved.
+ */
+int rcx_debug_inject_wait_timeout(int64_t spins);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RCX_H */

@@ -1,0 +1,748 @@
+// Tensor-core (tcgen05 / TMEM / TMA) blockwise causal attention, bf16, d = 128.
+//
+// What it computes is the FlashAttention recipe of the "Context Extension"
+// concept page (FlashAttention section): Q, K, V cut into B_r x B_c tiles kept
+// on chip, S = QK^T per tile, an online softmax with a running max, O
+// accumulated tile by tile, no n x n matrix in HBM -- with the RoPE rotation of
+// Q folded into the Q tile load ("Technical principles" of the same page), a
+// causal / sliding-window / sink mask ("Context window extension: 4K to 1M"
+// 4.1, 4.2), GQA, the YaRN temperature in the logit scale (same page 2.4) and
+// KV blocks visited in Ring-Attention order (same page 5.3).
+//
+// B200 design (one CTA per SM, 320 threads):
+//   warps 0-3  softmax for Q tile 0 (one thread per row; TMEM lanes 0-127)
+//   warps 4-7  softmax for Q tile 1
+//   warp  8    TMA producer: Q tiles once, then K and V tiles through a
+//              two-stage ring of 128B-swizzled shared-memory buffers
+//   warp  9    MMA issuer (one thread) and TMEM owner
+// TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1, 128 columns each.
+// The softmax writes P as packed bf16 over the first 64 columns of its S, and
+// O += P V reads P straight from TMEM (the .kind::f16 form with A in TMEM).
+// The two Q tiles of a CTA are two query heads of one GQA group over the same
+// 128 rows (so both read the same K/V tiles and share one mask), or, for an
+// odd group size, rows r and r + 128 of one head.
+// Rescaling of O is lazy: the reference max only moves when the row max grows
+// by more than 2^8, so most tiles skip the TMEM round trip of O.
+// Every mbarrier wait is bounded (about one second); on expiry the kernel
+// records RCX_ERR_DEVICE_TIMEOUT, raises a CTA-wide abort flag, lets its own
+// TMA copies and MMAs drain, frees TMEM and returns.
+#pragma once
+#include <cudaTypedefs.h>
+#include "attn_common.cuh"
+
+namespace rcx {
+
+constexpr int kTcBM = 128;          // query rows per Q tile
+constexpr int kTcBN = 128;          // keys per KV tile
+constexpr int kTcD = 128;           // head dim
+constexpr int kTcStages = 2;        // K/V pipeline depth
+constexpr int kTcThreads = 320;
+constexpr uint32_t kTileBytes = kTcBM * kTcD * 2;   // 32 KB bf16 tile
+constexpr uint32_t kHalfTileBytes = kTileBytes / 2; // one 64-column swizzled block
+constexpr float kLazyRescale = 8.0f;                // log2 units
+constexpr uint64_t kWaitLimitNs = 1000000000ull;    // one second
+
+struct TcParams {
+  AttnArgs a;
+  int pair_heads;        // 1: slots are heads h, h+1 over the same rows; 0: rows r, r+128 of one head
+  int n_rb;              // row blocks per (batch, head-or-pair)
+  int n_hg;              // heads (or head pairs) per batch
+  int64_t inject_spins;  // test hook: wait this long on a barrier nobody signals
+};
+
+// Shared-memory layout (offsets from a 1024-byte aligned base).
+constexpr uint32_t kSmQ = 0;                                  // 2 Q tiles
+constexpr uint32_t kSmK = kSmQ + 2 * kTileBytes;              // stages of K
+constexpr uint32_t kSmV = kSmK + kTcStages * kTileBytes;      // stages of V
+constexpr uint32_t kSmBar = kSmV + kTcStages * kTileBytes;    // barriers
+constexpr uint32_t kSmTotal = kSmBar + 256 + 1024;            // + alignment slack
+
+// ------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait.  Returns false when the CTA is aborting or the limit passed
+// (the latter records the timeout and raises the abort flag).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       uint64_t limit_ns = kWaitLimitNs, bool honour_abort = true) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 31) == 0) {
+      if (honour_abort && *abort_flag) return false;
+      if (global_timer() - t0 > limit_ns) {
+        if (honour_abort) {
+          *abort_flag = 1;
+          record_device_error(RCX_ERR_DEVICE_TIMEOUT);
+        }
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                              int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, shapes from the instruction descriptor.
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem].
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+#define RCX_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
+                  "=r"(r[i + 6]), "=r"(r[i + 7])
+#define RCX_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
+                  "r"(r[i + 6]), "r"(r[i + 7])
+
+// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : RCX_R8(0), RCX_R8(8), RCX_R8(16), RCX_R8(24)
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      RCX_W8(0), RCX_W8(8), RCX_W8(16), RCX_W8(24)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout
+// (start >> 4 at bit 0, leading byte offset >> 4 at 16, stride byte offset
+// >> 4 at 32, descriptor version 1 at bit 46, swizzle mode 2 at bit 61).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator,
+// M = 128, N = 128; b_mn_major selects an MN-major B (V, d contiguous).
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
+  return (1u << 4)                        // D format f32
+         | (1u << 7)                      // A format bf16
+         | (1u << 10)                     // B format bf16
+         | ((b_mn_major ? 1u : 0u) << 16) // B major
+         | ((uint32_t)(kTcBN >> 3) << 17) // N / 8
+         | ((uint32_t)(kTcBM >> 4) << 24);// M / 16
+}
+
+// ------------------------------------------------------------ tile walk
+
+// KV tiles (128 keys, local index t covers keys k_start + 128 t ...) that a
+// pair of Q tiles may see, in Ring-Attention block order: the block holding
+// the query rows first, then the blocks below it, then (wrapping) the blocks
+// above.  Visible tiles are the window/causal range [main_lo, main_hi] and
+// the sink tiles [0, sink_hi].
+struct TileWalk {
+  int main_lo, main_hi, sink_hi, top;
+  int64_t k0, kvb;
+  int64_t blk, blk_min, blk_max, blk_start;
+  int cur, phase;
+};
+
+__device__ __forceinline__ int64_t tw_block_of(const TileWalk& w, int t) { return (w.k0 + (int64_t)t * kTcBN) / w.kvb; }
+
+__device__ __forceinline__ int tw_first_tile(const TileWalk& w, int64_t blk) {
+  const int64_t x = blk * w.kvb - w.k0;
+  return x <= 0 ? 0 : (int)((x + kTcBN - 1) / kTcBN);
+}
+
+__device__ void tw_init(TileWalk& w, int64_t i_lo, int64_t i_hi, const AttnArgs& a) {
+  const int64_t Nk = a.k.N;
+  const int64_t key_end = a.k_start + Nk;
+  w.k0 = a.k_start;
+  w.kvb = a.kv_block;
+  w.main_lo = 0x3fffffff;
+  w.main_hi = -1;
+  w.sink_hi = -1;
+  w.phase = 2;
+  w.cur = -1;
+  const int64_t a1 = min(i_hi, key_end - 1) - a.k_start;                 // last causal key (local)
+  if (a1 < 0) return;
+  const int64_t a0 = a.window > 0 ? max(i_lo - a.window + 1 - a.k_start, (int64_t)0) : 0;
+  if (a0 <= a1) {
+    w.main_lo = (int)(a0 / kTcBN);
+    w.main_hi = (int)(a1 / kTcBN);
+  }
+  if (a.window > 0 && a.n_sink > a.k_start) {
+    const int64_t s_last = min(min(a.n_sink - a.k_start, Nk) - 1, a1);   // last sink key (local)
+    if (s_last >= 0) w.sink_hi = min((int)(s_last / kTcBN), w.main_lo - 1);
+  }
+  w.top = w.main_hi >= w.main_lo ? w.main_hi : w.sink_hi;
+  if (w.top < 0) return;
+  w.blk_min = tw_block_of(w, 0);
+  w.blk_max = tw_block_of(w, w.top);
+  w.blk_start = min(max(i_lo / w.kvb, w.blk_min), w.blk_max);
+  w.blk = w.blk_start;
+  w.phase = 0;
+}
+
+__device__ bool tw_next(TileWalk& w, int& tile) {
+  while (w.phase < 2) {
+    const int first = tw_first_tile(w, w.blk);
+    const int last = min(tw_first_tile(w, w.blk + 1) - 1, w.top);
+    int c = max(w.cur, first);
+    if (c > w.sink_hi && c < w.main_lo) c = w.main_lo;
+    if (c <= last) {
+      tile = c;
+      w.cur = c + 1;
+      return true;
+    }
+    w.cur = -1;
+    if (w.phase == 0) {
+      if (w.blk > w.blk_min) {
+        --w.blk;
+      } else {
+        w.phase = 1;
+        w.blk = w.blk_max;
+        if (w.blk <= w.blk_start) w.phase = 2;
+      }
+    } else {
+      if (w.blk - 1 > w.blk_start) --w.blk;
+      else w.phase = 2;
+    }
+  }
+  return false;
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <typename Tout>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ TcParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const AttnArgs& a = P.a;
+
+  // barriers
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmBar);
+  const uint32_t bar0 = smem_addr(bars);
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  enum {
+    B_QFULL = 0,      // [2]
+    B_QREADY = 2,     // [2]
+    B_KFULL = 4,      // [stages]
+    B_KEMPTY = 4 + kTcStages,
+    B_VFULL = 4 + 2 * kTcStages,
+    B_VEMPTY = 4 + 3 * kTcStages,
+    B_SFULL = 4 + 4 * kTcStages,  // [2]
+    B_PREADY = B_SFULL + 2,       // [2]
+    B_OFINAL = B_PREADY + 2,      // [2]
+    B_DRAIN = B_OFINAL + 2,
+    B_NEVER = B_DRAIN + 1,
+    B_COUNT = B_NEVER + 1
+  };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmBar + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmBar + 8 * B_COUNT + 8);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- work item: (row block, head group, batch), heaviest row blocks first
+  const int item = blockIdx.x;
+  const int per_rb = P.n_hg * (int)a.q.B;
+  const int rb = P.n_rb - 1 - item / per_rb;
+  const int hg = (item % per_rb) % P.n_hg;
+  const int64_t bb = (item % per_rb) / P.n_hg;
+  int head[2];
+  int64_t row0[2];
+  if (P.pair_heads) {
+    head[0] = 2 * hg; head[1] = 2 * hg + 1;
+    row0[0] = row0[1] = (int64_t)rb * kTcBM;
+  } else {
+    head[0] = head[1] = hg;
+    row0[0] = (int64_t)rb * 2 * kTcBM;
+    row0[1] = row0[0] + kTcBM;
+  }
+  const int kvh = head[0] / a.G;
+  const int64_t Nq = a.q.N;
+  // global row range covered by real rows of the two tiles
+  const int64_t gi_lo = a.q_start + row0[0];
+  const int64_t gi_hi = a.q_start + min(max(row0[0], row0[1]) + kTcBM, Nq) - 1;
+  const int64_t key_end = a.k_start + a.k.N;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < B_COUNT; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_QREADY || i == B_QREADY + 1 || i == B_PREADY || i == B_PREADY + 1) cnt = kTcBM;
+      mbar_init(BAR(i), cnt);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) tmem_alloc(smem_addr(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem + 0, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 384};
+
+  if (warp == 8) {
+    // ================================================================ producer
+    if (lane == 0) {
+      for (int s = 0; s < 2; ++s) {
+        mbar_expect_tx(BAR(B_QFULL + s), kTileBytes);
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_tile(sbase + kSmQ + s * kTileBytes + kb * kHalfTileBytes, &tm_q, BAR(B_QFULL + s), kb * 64,
+                        head[s], (int)row0[s], (int)bb);
+      }
+      TileWalk w;
+      tw_init(w, gi_lo, gi_hi, a);
+      int tile, jt = 0;
+      int issued[kTcStages];
+      for (int s = 0; s < kTcStages; ++s) issued[s] = 0;
+      while (tw_next(w, tile)) {
+        const int st = jt % kTcStages;
+        const uint32_t par = ((jt / kTcStages) & 1) ^ 1;
+        if (!mbar_wait(BAR(B_KEMPTY + st), par, abort_flag)) break;
+        mbar_expect_tx(BAR(B_KFULL + st), kTileBytes);
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_tile(sbase + kSmK + st * kTileBytes + kb * kHalfTileBytes, &tm_k, BAR(B_KFULL + st), kb * 64,
+                        kvh, tile * kTcBN, (int)bb);
+        if (!mbar_wait(BAR(B_VEMPTY + st), par, abort_flag)) {
+          issued[st] = 2 * (jt / kTcStages) + 1;   // K of this use issued, V not
+          break;
+        }
+        mbar_expect_tx(BAR(B_VFULL + st), kTileBytes);
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_tile(sbase + kSmV + st * kTileBytes + kb * kHalfTileBytes, &tm_v, BAR(B_VFULL + st), kb * 64,
+                        kvh, tile * kTcBN, (int)bb);
+        issued[st] = 2 * (jt / kTcStages) + 2;
+        ++jt;
+      }
+      if (*abort_flag) {
+        // drain: wait (bounded, ignoring the abort flag) for copies in flight
+        for (int s = 0; s < 2; ++s) mbar_wait(BAR(B_QFULL + s), 0, abort_flag, 100000000ull, false);
+        for (int st = 0; st < kTcStages; ++st) {
+          if (issued[st] == 0) continue;
+          const int use = (issued[st] - 1) / 2;
+          mbar_wait(BAR(B_KFULL + st), use & 1, abort_flag, 100000000ull, false);
+          if (issued[st] % 2 == 0) mbar_wait(BAR(B_VFULL + st), use & 1, abort_flag, 100000000ull, false);
+        }
+      }
+    }
+    __syncwarp();   // reconverge before the CTA-wide barrier
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      if (P.inject_spins > 0) {
+        // test hook: a wait that nothing ends
+        bool got = false;
+        for (int64_t i = 0; i < P.inject_spins && !got; ++i) got = mbar_test(BAR(B_NEVER), 0);
+        if (!got) {
+          *abort_flag = 1;
+          record_device_error(RCX_ERR_DEVICE_TIMEOUT);
+          ok = false;
+        }
+      }
+      TileWalk w;
+      tw_init(w, gi_lo, gi_hi, a);
+      int n = 0, tile;
+      while (tw_next(w, tile)) ++n;
+      constexpr uint32_t id_qk = idesc_bf16(false);
+      constexpr uint32_t id_pv = idesc_bf16(true);
+      ok = ok && mbar_wait(BAR(B_QREADY + 0), 0, abort_flag) && mbar_wait(BAR(B_QREADY + 1), 0, abort_flag);
+      auto issue_s = [&](int s, int st) {
+        const uint32_t qa = sbase + kSmQ + s * kTileBytes;
+        const uint32_t ka = sbase + kSmK + st * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcD / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kHalfTileBytes + (kk % 4) * 32;
+          umma_ss(tS[s], sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int s, int st, bool first_tile) {
+        const uint32_t va = sbase + kSmV + st * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcBN / 16; ++kk)
+          umma_ts(tO[s], tS[s] + kk * 8, sw128_desc(va + kk * 2048, kHalfTileBytes, 1024), id_pv,
+                  (!first_tile || kk > 0) ? 1u : 0u);
+      };
+      if (ok && n > 0) {
+        ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          umma_commit(BAR(B_SFULL + 0));
+          issue_s(1, 0);
+          umma_commit(BAR(B_SFULL + 1));
+          umma_commit(BAR(B_KEMPTY + 0));
+        }
+        for (int jt = 0; ok && jt < n; ++jt) {
+          const int st = jt % kTcStages;
+          const uint32_t par = (jt / kTcStages) & 1;
+          const bool last = jt == n - 1;
+          const int st1 = (jt + 1) % kTcStages;
+          const uint32_t par1 = ((jt + 1) / kTcStages) & 1;
+          if (!(ok = mbar_wait(BAR(B_VFULL + st), par, abort_flag))) break;
+          if (!(ok = mbar_wait(BAR(B_PREADY + 0), jt & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(0, st, jt == 0);
+          if (last) umma_commit(BAR(B_OFINAL + 0));
+          if (!last) {
+            if (!(ok = mbar_wait(BAR(B_KFULL + st1), par1, abort_flag))) break;
+            tc_fence_after();
+            issue_s(0, st1);
+            umma_commit(BAR(B_SFULL + 0));
+          }
+          if (!(ok = mbar_wait(BAR(B_PREADY + 1), jt & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(1, st, jt == 0);
+          umma_commit(BAR(B_VEMPTY + st));
+          if (last) umma_commit(BAR(B_OFINAL + 1));
+          if (!last) {
+            issue_s(1, st1);
+            umma_commit(BAR(B_SFULL + 1));
+            umma_commit(BAR(B_KEMPTY + st1));
+          }
+        }
+      }
+      // all MMAs this thread issued complete before TMEM is released
+      umma_commit(BAR(B_DRAIN));
+      mbar_wait(BAR(B_DRAIN), 0, abort_flag, 100000000ull, false);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax
+    const int s = warp / 4;                 // Q tile (slot) of this warpgroup
+    const int q4 = warp % 4;                // TMEM lane quarter
+    const int r = q4 * 32 + lane;           // row within the tile
+    const int64_t row = row0[s] + r;        // local q row
+    const int64_t gi = a.q_start + row;     // global token index
+    const bool row_ok = row < Nq;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_QFULL + s), 0, abort_flag));
+
+    // Rotate this row of the Q tile in shared memory (fused RoPE on Q).
+    if (ok && (a.rope_flags & RCX_ROTATE_Q) && row_ok) {
+      const int64_t m = a.positions ? a.positions[gi] : gi;
+      uint8_t* qrow = smem + kSmQ + s * kTileBytes + r * 128;
+#pragma unroll 1
+      for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* p = reinterpret_cast<uint4*>(qrow + kb * kHalfTileBytes + ((c ^ (r & 7)) * 16));
+          uint4 u = *p;
+          uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float cs, sn;
+            rope_cos_sin(m, a.f.theta[kb * 32 + c * 4 + e], cs, sn);
+            const float2 x = bf2_to_f2(wv[e]);
+            wv[e] = f2_to_bf2(x.x * cs - x.y * sn, x.x * sn + x.y * cs);
+          }
+          *p = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    mbar_arrive(BAR(B_QREADY + s));
+
+    TileWalk w;
+    tw_init(w, gi_lo, gi_hi, a);
+    const int64_t ti_lo = a.q_start + row0[s], ti_hi = ti_lo + kTcBM - 1;
+    float m_used = -INFINITY, l = 0.f;
+    int tile, jt = 0;
+    while (ok && tw_next(w, tile)) {
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + s), jt & 1, abort_flag)))) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tS[s] + lane_off + 0, sr);
+      tmem_ld32(tS[s] + lane_off + 32, sr + 32);
+      tmem_ld32(tS[s] + lane_off + 64, sr + 64);
+      tmem_ld32(tS[s] + lane_off + 96, sr + 96);
+      tmem_wait_ld();
+      const int64_t j0 = a.k_start + (int64_t)tile * kTcBN;
+      const bool full = (j0 + kTcBN <= key_end) &&
+                        tile_all_visible(ti_lo, ti_hi, j0, j0 + kTcBN - 1, a.window, a.n_sink);
+      float mx = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      } else {
+        // The mask of this row over columns c of the tile, in 32-bit form:
+        // c <= lim (causal and inside the keys) and (c > win_lo or c <= snk).
+        auto clip = [](int64_t x) { return (int)(x < -1 ? -1 : (x > kTcBN ? kTcBN : x)); };
+        const int lim = clip(min(gi, key_end - 1) - j0);
+        const int win_lo = a.window > 0 ? clip(gi - a.window - j0) : -1;
+        const int snk = a.window > 0 ? clip(a.n_sink - 1 - j0) : -1;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const bool vis = c <= lim && (c > win_lo || c <= snk);
+          if (!vis) sr[c] = __float_as_uint(-INFINITY);
+          mx = fmaxf(mx, __uint_as_float(sr[c]));
+        }
+      }
+      const float m_new = fmaxf(m_used, mx * a.scale_log2);
+      const bool need = m_new > m_used + kLazyRescale;
+      float alpha = 1.f;
+      if (need) {
+        alpha = fast_exp2(m_used - m_new);   // 0 when m_used = -inf
+        m_used = m_new;
+        l *= alpha;
+      }
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), a.scale_log2, -mref));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), a.scale_log2, -mref));
+        sum += p0 + p1;
+        pk[c] = f2_to_bf2(p0, p1);
+      }
+      l += sum;
+      tmem_st32(tS[s] + lane_off + 0, pk);
+      tmem_st32(tS[s] + lane_off + 32, pk + 32);
+      if (__any_sync(0xffffffffu, need && jt > 0)) {
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t o[32];
+          tmem_ld32(tO[s] + lane_off + cb * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tO[s] + lane_off + cb * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(B_PREADY + s));
+      ++jt;
+    }
+
+    // ---- epilogue: O / l -> global, LSE
+    if (ok) {
+      const int n_tiles = jt;
+      if (n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_OFINAL + s), 0, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        Tout* op = reinterpret_cast<Tout*>(a.o.ptr) + bb * a.o.sb + row * a.o.sn + head[s] * a.o.sh;
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t o[32];
+          if (n_tiles > 0) {
+            tmem_ld32(tO[s] + lane_off + cb * 32, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = 0u;
+          }
+          if (row_ok) {
+            if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 8) {
+                uint4 v;
+                v.x = f2_to_bf2(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
+                v.y = f2_to_bf2(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                v.z = f2_to_bf2(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
+                v.w = f2_to_bf2(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
+                *reinterpret_cast<uint4*>(op + cb * 32 + c) = v;
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; c += 4) {
+                float4 v = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
+                                       __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
+                *reinterpret_cast<float4*>(op + cb * 32 + c) = v;
+              }
+            }
+          }
+        }
+        if (row_ok && a.lse)
+          a.lse[bb * a.lse_sb + head[s] * a.lse_sh + row] =
+              l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host side
+
+static int64_t g_tc_inject_spins = 0;
+inline void attn_tc_set_inject(int64_t spins) { g_tc_inject_spins = spins; }
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D map over a [B, N, H, 128] bf16 view, box = 64 columns x 1 head x 128 tokens.
+static int make_tile_map(CUtensorMap* map, const rcx_tensor& t) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return RCX_ERR_CUDA;
+  const int64_t B = t.shape[0], N = t.shape[1], H = t.shape[2], D = t.shape[3];
+  // Unit-size dimensions get a dense stride (TMA wants 16-byte multiples).
+  const int64_t sh = H > 1 ? t.stride[2] : D;
+  const int64_t sn = N > 1 ? t.stride[1] : sh * H;
+  const int64_t sb = B > 1 ? t.stride[0] : sn * N;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(sn * 2), (cuuint64_t)(sb * 2)};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)kTcBM, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.ptr, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RCX_OK : RCX_ERR_CUDA;
+}
+
+static bool tc_view_ok(const rcx_tensor& t) {
+  if (t.dtype != RCX_BF16 || t.shape[3] != kTcD) return false;
+  if (reinterpret_cast<uintptr_t>(t.ptr) % 16) return false;
+  for (int i = 0; i < 3; ++i)
+    if (t.stride[i] % 8) return false;
+  if (t.shape[1] > 0x7fffffff - 2 * kTcBM || t.shape[2] > 0x7fffffff || t.shape[0] > 0x7fffffff) return false;
+  return true;
+}
+
+static int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v,
+                          const rcx_tensor& o, cudaStream_t stream) {
+  if (!tc_view_ok(q) || !tc_view_ok(k) || !tc_view_ok(v)) return RCX_ERR_ALIGNMENT;
+  const int oes = o.dtype == RCX_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(o.ptr) % 16 || o.stride[0] % (16 / oes) || o.stride[1] % (16 / oes) ||
+      o.stride[2] % (16 / oes))
+    return RCX_ERR_ALIGNMENT;
+  if (a.k.N == 0) {
+    // no keys at all: every row is empty -> handled by the kernel (zero tiles)
+  }
+  CUtensorMap mq, mk, mv;
+  int st;
+  if ((st = make_tile_map(&mq, q)) || (st = make_tile_map(&mk, k)) || (st = make_tile_map(&mv, v))) return st;
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.a = a;
+  p.pair_heads = (a.G % 2 == 0) ? 1 : 0;
+  const int64_t rows_per_item = p.pair_heads ? kTcBM : 2 * kTcBM;
+  p.n_rb = (int)((a.q.N + rows_per_item - 1) / rows_per_item);
+  p.n_hg = (int)(p.pair_heads ? a.q.H / 2 : a.q.H);
+  p.inject_spins = g_tc_inject_spins;
+  const int64_t items = (int64_t)p.n_rb * p.n_hg * a.q.B;
+  if (items <= 0) return RCX_OK;
+  if (items > 0x7fffffff) return RCX_ERR_UNSUPPORTED;
+  if (o.dtype == RCX_BF16) {
+    cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+    attn_tc_kernel<__nv_bfloat16><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
+  } else {
+    cudaFuncSetAttribute(attn_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+    attn_tc_kernel<float><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RCX_OK : RCX_ERR_CUDA;
+}
+
+}  // namespace rcx

@@ -1,0 +1,523 @@
+// librcx.so: the C ABI declared in include/rcx.h.
+//
+// One translation unit: host-side argument checks, launch configuration, the
+// Ring-Attention schedule and the host float64 frequency schedules; the
+// kernels live in the *.cuh files included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "rope_apply.cuh"
+#include "merge.cuh"
+#include "attn_common.cuh"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+#include "rope_freqs.inc"
+
+using namespace rcx;
+
+namespace {
+
+constexpr int kAbiVersion = 100;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline int elem_size(int dtype) { return dtype == RCX_BF16 ? 2 : 4; }
+
+bool shape_ok(const rcx_tensor& t) {
+  for (int i = 0; i < 4; ++i)
+    if (t.shape[i] < 0) return false;
+  return t.dtype == RCX_F32 || t.dtype == RCX_BF16;
+}
+
+// [B, N, H, d] activation view: unit stride on d, non-negative strides.
+int check_act(const rcx_tensor& t) {
+  if (!shape_ok(t)) return RCX_ERR_INVALID_ARG;
+  const bool empty = t.shape[0] == 0 || t.shape[1] == 0 || t.shape[2] == 0 || t.shape[3] == 0;
+  if (!t.ptr && !empty) return RCX_ERR_INVALID_ARG;
+  if (!t.ptr && t.shape[0] == 0 && t.shape[3] == 0) return RCX_ERR_INVALID_ARG;   // an all-zero (null) view
+  if (t.stride[3] != 1 || t.stride[0] < 0 || t.stride[1] < 0 || t.stride[2] < 0) return RCX_ERR_INVALID_ARG;
+  return RCX_OK;
+}
+
+// 16-byte vector access along d: base and token/head/batch strides aligned.
+bool vec16_ok(const rcx_tensor& t) {
+  const int es = elem_size(t.dtype);
+  const int per = 16 / es;
+  if (reinterpret_cast<uintptr_t>(t.ptr) % 16) return false;
+  if (t.shape[3] % per) return false;
+  for (int i = 0; i < 3; ++i)
+    if (t.stride[i] % per) return false;
+  return true;
+}
+
+// [B, H, N, 1] fp32 LSE view with unit stride on N.
+int check_lse(const rcx_tensor& t, int64_t B, int64_t H, int64_t N) {
+  if (!t.ptr && B * H * N != 0) return RCX_ERR_INVALID_ARG;
+  if (t.dtype != RCX_F32) return RCX_ERR_INVALID_ARG;
+  if (t.shape[0] != B || t.shape[1] != H || t.shape[2] != N) return RCX_ERR_INVALID_ARG;
+  if (t.stride[2] != 1 || t.stride[0] < 0 || t.stride[1] < 0) return RCX_ERR_INVALID_ARG;
+  return RCX_OK;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "librcx: launch failed: %s\n", cudaGetErrorString(e));
+    return RCX_ERR_CUDA;
+  }
+  return RCX_OK;
+}
+
+rcx_tensor null_tensor() {
+  rcx_tensor t;
+  std::memset(&t, 0, sizeof(t));
+  return t;
+}
+
+// Sub-view of tokens [n0, n0 + n) of a [B, N, H, d] tensor.
+rcx_tensor token_slice(const rcx_tensor& t, int64_t n0, int64_t n) {
+  rcx_tensor s = t;
+  s.ptr = static_cast<char*>(t.ptr) + n0 * t.stride[1] * elem_size(t.dtype);
+  s.shape[1] = n;
+  return s;
+}
+
+// Sub-view of tokens [n0, n0 + n) of a [B, H, N, 1] LSE tensor.
+rcx_tensor lse_slice(const rcx_tensor& t, int64_t n0, int64_t n) {
+  rcx_tensor s = t;
+  s.ptr = static_cast<char*>(t.ptr) + n0 * 4;
+  s.shape[2] = n;
+  return s;
+}
+
+rcx_tensor make_tensor(void* p, int dtype, int64_t B, int64_t N, int64_t H, int64_t D) {
+  rcx_tensor t;
+  t.ptr = p;
+  t.dtype = dtype;
+  t.shape[0] = B; t.shape[1] = N; t.shape[2] = H; t.shape[3] = D;
+  t.stride[3] = 1; t.stride[2] = D; t.stride[1] = H * D; t.stride[0] = N * H * D;
+  return t;
+}
+
+rcx_tensor make_lse(void* p, int64_t B, int64_t H, int64_t N) {
+  rcx_tensor t;
+  t.ptr = p;
+  t.dtype = RCX_F32;
+  t.shape[0] = B; t.shape[1] = H; t.shape[2] = N; t.shape[3] = 1;
+  t.stride[3] = 1; t.stride[2] = 1; t.stride[1] = N; t.stride[0] = H * N;
+  return t;
+}
+
+// ------------------------------------------------------------------ rope_apply
+
+int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& q_out,
+                    const rcx_tensor& k_out, const int64_t* positions, int64_t n_positions,
+                    const double* inv_freq, cudaStream_t stream) {
+  if (!inv_freq) return RCX_ERR_INVALID_ARG;
+  const bool has_q = q.ptr != nullptr, has_k = k.ptr != nullptr;
+  if (!has_q && !has_k) return RCX_OK;
+  const rcx_tensor& ref = has_q ? q : k;
+  const int dtype = ref.dtype;
+  const int64_t B = ref.shape[0], N = ref.shape[1], D = ref.shape[3];
+  if (D < 2 || D > 2 * kMaxPairs || (D & 1)) return RCX_ERR_INVALID_ARG;
+  const rcx_tensor* ins[2] = {&q, &k};
+  const rcx_tensor* outs[2] = {&q_out, &k_out};
+  for (int i = 0; i < 2; ++i) {
+    if (!ins[i]->ptr) continue;
+    int st = check_act(*ins[i]);
+    if (st) return st;
+    st = check_act(*outs[i]);
+    if (st) return st;
+    if (ins[i]->dtype != dtype || outs[i]->dtype != dtype) return RCX_ERR_INVALID_ARG;
+    if (ins[i]->shape[0] != B || ins[i]->shape[1] != N || ins[i]->shape[3] != D) return RCX_ERR_INVALID_ARG;
+    for (int j = 0; j < 4; ++j)
+      if (outs[i]->shape[j] != ins[i]->shape[j]) return RCX_ERR_INVALID_ARG;
+    if (!vec16_ok(*ins[i]) || !vec16_ok(*outs[i])) return RCX_ERR_ALIGNMENT;
+  }
+  if (positions && n_positions < N) return RCX_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return RCX_OK;
+  RopeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (has_q) { a.q_in = make_view(q); a.q_out = make_view(q_out); }
+  if (has_k) { a.k_in = make_view(k); a.k_out = make_view(k_out); }
+  a.positions = positions;
+  a.n_tok = B * N;
+  a.N = N;
+  a.pairs = (int)(D / 2);
+  for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
+  const int64_t groups = (a.n_tok + kRopeTok - 1) / kRopeTok;
+  const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 8);
+  if (dtype == RCX_BF16)
+    rope_apply_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, stream>>>(a);
+  else
+    rope_apply_kernel<float><<<grid, kRopeThreads, 0, stream>>>(a);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------- merge
+
+int merge_impl(const rcx_tensor& oa, const rcx_tensor& la, const rcx_tensor& ob, const rcx_tensor& lb,
+               const rcx_tensor& oo_in, const rcx_tensor& lo_in, cudaStream_t stream) {
+  const bool in_place = oo_in.ptr == nullptr;
+  const rcx_tensor& oo = in_place ? oa : oo_in;
+  const rcx_tensor& lo = in_place ? la : lo_in;
+  int st;
+  if ((st = check_act(oa)) || (st = check_act(ob)) || (st = check_act(oo))) return st;
+  if (oa.dtype != RCX_F32 || ob.dtype != RCX_F32) return RCX_ERR_INVALID_ARG;
+  const int64_t B = oa.shape[0], N = oa.shape[1], H = oa.shape[2], D = oa.shape[3];
+  for (int j = 0; j < 4; ++j)
+    if (ob.shape[j] != oa.shape[j] || oo.shape[j] != oa.shape[j]) return RCX_ERR_INVALID_ARG;
+  if ((st = check_lse(la, B, H, N)) || (st = check_lse(lb, B, H, N)) || (st = check_lse(lo, B, H, N)))
+    return st;
+  if (D < 4 || D > 128 || (D & (D - 1))) return RCX_ERR_UNSUPPORTED;   // d/4 must divide 32
+  if (!vec16_ok(oa) || !vec16_ok(ob)) return RCX_ERR_ALIGNMENT;
+  if (oo.dtype == RCX_BF16 ? (reinterpret_cast<uintptr_t>(oo.ptr) % 8 || oo.stride[0] % 4 ||
+                              oo.stride[1] % 4 || oo.stride[2] % 4)
+                           : !vec16_ok(oo))
+    return RCX_ERR_ALIGNMENT;
+  if (B == 0 || N == 0 || H == 0) return RCX_OK;
+  MergeArgs a;
+  a.oa = make_view(oa); a.ob = make_view(ob); a.oo = make_view(oo);
+  a.la = static_cast<float*>(la.ptr); a.lb = static_cast<const float*>(lb.ptr);
+  a.lo = static_cast<float*>(lo.ptr);
+  a.la_sb = la.stride[0]; a.la_sh = la.stride[1];
+  a.lb_sb = lb.stride[0]; a.lb_sh = lb.stride[1];
+  a.lo_sb = lo.stride[0]; a.lo_sh = lo.stride[1];
+  a.rows = B * N * H;
+  a.d4 = (int)(D / 4);
+  const int64_t warps = (a.rows * a.d4 + 31) / 32;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 16));
+  if (oo.dtype == RCX_BF16)
+    merge_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
+  else
+    merge_kernel<float><<<grid, 256, 0, stream>>>(a);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ attention
+
+template <typename T, typename Tout>
+int launch_simt(const AttnArgs& a, cudaStream_t stream) {
+  const int64_t D = a.q.D;
+  const int64_t tiles = (a.q.N + kSimtBR - 1) / kSimtBR;
+  dim3 grid((unsigned)tiles, (unsigned)a.q.H, (unsigned)a.q.B);
+  const size_t smem = (size_t)2 * kSimtBC * D * sizeof(float);
+  if (D == 32) {
+    cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_simt_kernel<T, Tout, 1><<<grid, kSimtBR * 1, smem, stream>>>(a);
+  } else if (D == 64) {
+    cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_simt_kernel<T, Tout, 2><<<grid, kSimtBR * 2, smem, stream>>>(a);
+  } else {
+    cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_simt_kernel<T, Tout, 4><<<grid, kSimtBR * 4, smem, stream>>>(a);
+  }
+  return launch_status();
+}
+
+int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, const rcx_tensor& o,
+              const rcx_tensor& lse, int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+              int64_t q_start, int64_t k_start, const int64_t* positions, int64_t n_positions,
+              const double* inv_freq, int rope_flags, cudaStream_t stream) {
+  int st;
+  if ((st = check_act(q)) || (st = check_act(k)) || (st = check_act(v)) || (st = check_act(o))) return st;
+  const int64_t B = q.shape[0], Nq = q.shape[1], Hq = q.shape[2], D = q.shape[3];
+  const int64_t Nk = k.shape[1], Hkv = k.shape[2];
+  if (k.shape[0] != B || v.shape[0] != B || o.shape[0] != B) return RCX_ERR_INVALID_ARG;
+  if (k.shape[3] != D || v.shape[3] != D || o.shape[3] != D) return RCX_ERR_INVALID_ARG;
+  if (v.shape[1] != Nk || v.shape[2] != Hkv || o.shape[1] != Nq || o.shape[2] != Hq) return RCX_ERR_INVALID_ARG;
+  if (Hkv <= 0 || Hq <= 0 || Hq % Hkv) return RCX_ERR_INVALID_ARG;
+  if (q.dtype != k.dtype || q.dtype != v.dtype) return RCX_ERR_INVALID_ARG;
+  if (lse.ptr && (st = check_lse(lse, B, Hq, Nq))) return st;
+  if (kv_block < 0 || window < 0 || n_sink < 0 || q_start < 0 || k_start < 0) return RCX_ERR_INVALID_ARG;
+  if (!(temperature > 0.0) || !std::isfinite(temperature)) return RCX_ERR_INVALID_ARG;
+  if (rope_flags & ~(RCX_ROTATE_Q | RCX_ROTATE_K)) return RCX_ERR_INVALID_ARG;
+  if (rope_flags && !inv_freq) return RCX_ERR_INVALID_ARG;
+  if (rope_flags && positions && n_positions < std::max(q_start + Nq, k_start + Nk)) return RCX_ERR_INVALID_ARG;
+  if (D < 2 || (D & 1)) return RCX_ERR_INVALID_ARG;
+  if (B == 0 || Nq == 0) return RCX_OK;
+
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = make_view(q); a.k = make_view(k); a.v = make_view(v); a.o = make_view(o);
+  a.lse = static_cast<float*>(lse.ptr);
+  a.lse_sb = lse.ptr ? lse.stride[0] : 0;
+  a.lse_sh = lse.ptr ? lse.stride[1] : 0;
+  a.q_start = q_start; a.k_start = k_start;
+  a.kv_block = kv_block > 0 ? kv_block : (k_start + Nk > 0 ? k_start + Nk : 1);
+  a.window = window; a.n_sink = n_sink;
+  a.scale_log2 = (float)(1.4426950408889634074 / (std::sqrt((double)D) * temperature));
+  a.positions = positions;
+  a.rope_flags = rope_flags;
+  a.pairs = (int)(D / 2);
+  a.G = (int)(Hq / Hkv);
+  if (rope_flags) {
+    if (a.pairs > kMaxPairs) return RCX_ERR_INVALID_ARG;
+    for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
+  }
+
+  if (q.dtype == RCX_BF16 && D == 128) {
+    if (rope_flags & RCX_ROTATE_K) return RCX_ERR_UNSUPPORTED;
+    return attn_tc_launch(a, q, k, v, o, stream);
+  }
+  if (D != 32 && D != 64 && D != 128) return RCX_ERR_UNSUPPORTED;
+  if (q.dtype == RCX_F32)
+    return o.dtype == RCX_F32 ? launch_simt<float, float>(a, stream) : launch_simt<float, __nv_bfloat16>(a, stream);
+  return o.dtype == RCX_F32 ? launch_simt<__nv_bfloat16, float>(a, stream)
+                            : launch_simt<__nv_bfloat16, __nv_bfloat16>(a, stream);
+}
+
+// ----------------------------------------------------------------------- ring
+
+struct RingPlan {
+  int64_t B, N, Hq, Hkv, D, kv, P;
+  bool rotate_k_separately;
+  int64_t off_acc, off_lacc, off_part, off_lpart, off_krot, total;
+};
+
+int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+RingPlan ring_plan(const rcx_tensor& q, const rcx_tensor& k, int64_t kv_block, int rope_flags) {
+  RingPlan p;
+  p.B = q.shape[0]; p.N = q.shape[1]; p.Hq = q.shape[2]; p.D = q.shape[3]; p.Hkv = k.shape[2];
+  p.kv = kv_block > 0 ? std::min(kv_block, std::max<int64_t>(p.N, 1)) : std::max<int64_t>(p.N, 1);
+  p.P = (p.N + p.kv - 1) / p.kv;
+  p.rotate_k_separately = (rope_flags & RCX_ROTATE_K) && q.dtype == RCX_BF16 && p.D == 128;
+  int64_t off = 0;
+  p.off_acc = off;   off = align256(off + p.B * p.N * p.Hq * p.D * 4);
+  p.off_lacc = off;  off = align256(off + p.B * p.Hq * p.N * 4);
+  p.off_part = off;  off = align256(off + p.B * p.kv * p.Hq * p.D * 4);
+  p.off_lpart = off; off = align256(off + p.B * p.Hq * p.kv * 4);
+  p.off_krot = off;
+  if (p.rotate_k_separately) off = align256(off + p.B * p.N * p.Hkv * p.D * 2);
+  p.total = off;
+  return p;
+}
+
+int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, const rcx_tensor& o,
+              const rcx_tensor& lse, int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+              const int64_t* positions, int64_t n_positions, const double* inv_freq, int rope_flags,
+              void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
+  int st;
+  if ((st = check_act(q)) || (st = check_act(k)) || (st = check_act(v)) || (st = check_act(o))) return st;
+  if (k.shape[1] != q.shape[1]) return RCX_ERR_INVALID_ARG;     // self-attention over one sequence
+  if (kv_block < 0) return RCX_ERR_INVALID_ARG;
+  RingPlan p = ring_plan(q, k, kv_block, rope_flags);
+  if (p.B == 0 || p.N == 0) return RCX_OK;
+  if (!workspace || workspace_bytes < p.total) return RCX_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return RCX_ERR_ALIGNMENT;
+  char* ws = static_cast<char*>(workspace);
+  rcx_tensor acc = make_tensor(ws + p.off_acc, RCX_F32, p.B, p.N, p.Hq, p.D);
+  rcx_tensor lacc = make_lse(ws + p.off_lacc, p.B, p.Hq, p.N);
+  rcx_tensor part = make_tensor(ws + p.off_part, RCX_F32, p.B, p.kv, p.Hq, p.D);
+  rcx_tensor lpart = make_lse(ws + p.off_lpart, p.B, p.Hq, p.kv);
+
+  rcx_tensor kk = k;
+  int flags = rope_flags;
+  if (p.rotate_k_separately) {
+    // K is shared by G query heads and by every query tile: rotate it once.
+    rcx_tensor krot = make_tensor(ws + p.off_krot, RCX_BF16, p.B, p.N, p.Hkv, p.D);
+    if ((st = rope_apply_impl(null_tensor(), k, null_tensor(), krot, positions, n_positions, inv_freq, stream)))
+      return st;
+    kk = krot;
+    flags &= ~RCX_ROTATE_K;
+  }
+
+  // Per shard: which ring steps carry visible keys (first and last).
+  std::vector<int64_t> first(p.P, -1), last(p.P, -1), count(p.P, 0);
+  for (int64_t t = 0; t < p.P; ++t)
+    for (int64_t r = 0; r < p.P; ++r) {
+      const int64_t b = ((r - t) % p.P + p.P) % p.P;
+      const int64_t i0 = r * p.kv, i1 = std::min((r + 1) * p.kv, p.N) - 1;
+      const int64_t j0 = b * p.kv, j1 = std::min((b + 1) * p.kv, p.N) - 1;
+      if (!tile_any_visible(i0, i1, j0, j1, window, n_sink)) continue;
+      if (first[r] < 0) first[r] = t;
+      last[r] = t;
+      ++count[r];
+    }
+
+  for (int64_t t = 0; t < p.P; ++t) {
+    for (int64_t r = 0; r < p.P; ++r) {
+      const int64_t b = ((r - t) % p.P + p.P) % p.P;
+      const int64_t i0 = r * p.kv, ni = std::min((r + 1) * p.kv, p.N) - i0;
+      const int64_t j0 = b * p.kv, nj = std::min((b + 1) * p.kv, p.N) - j0;
+      if (!tile_any_visible(i0, i0 + ni - 1, j0, j0 + nj - 1, window, n_sink)) continue;
+      rcx_tensor qs = token_slice(q, i0, ni);
+      rcx_tensor ks = token_slice(kk, j0, nj);
+      rcx_tensor vs = token_slice(v, j0, nj);
+      rcx_tensor os_final = token_slice(o, i0, ni);
+      rcx_tensor ls_final = lse.ptr ? lse_slice(lse, i0, ni) : null_tensor();
+      if (count[r] == 1) {          // one visible block: write the result directly
+        st = attn_impl(qs, ks, vs, os_final, ls_final, 0, window, n_sink, temperature, i0, j0, positions,
+                       n_positions, inv_freq, flags, stream);
+        if (st) return st;
+        continue;
+      }
+      rcx_tensor as = token_slice(acc, i0, ni);
+      rcx_tensor las = lse_slice(lacc, i0, ni);
+      if (t == first[r]) {
+        st = attn_impl(qs, ks, vs, as, las, 0, window, n_sink, temperature, i0, j0, positions, n_positions,
+                       inv_freq, flags, stream);
+        if (st) return st;
+        continue;
+      }
+      rcx_tensor ps = token_slice(part, 0, ni);
+      rcx_tensor lps = lse_slice(lpart, 0, ni);
+      st = attn_impl(qs, ks, vs, ps, lps, 0, window, n_sink, temperature, i0, j0, positions, n_positions,
+                     inv_freq, flags, stream);
+      if (st) return st;
+      if (t == last[r]) {
+        rcx_tensor lo = lse.ptr ? ls_final : las;
+        st = merge_impl(as, las, ps, lps, os_final, lo, stream);
+      } else {
+        st = merge_impl(as, las, ps, lps, null_tensor(), null_tensor(), stream);
+      }
+      if (st) return st;
+    }
+  }
+  return RCX_OK;
+}
+
+}  // namespace
+
+// =============================================================== C entry points
+
+extern "C" {
+
+int rcx_abi_version(void) { return kAbiVersion; }
+
+const char* rcx_status_string(int status) {
+  switch (status) {
+    case RCX_OK: return "ok";
+    case RCX_ERR_INVALID_ARG: return "invalid argument";
+    case RCX_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RCX_ERR_ALIGNMENT: return "misaligned pointer or stride";
+    case RCX_ERR_CUDA: return "CUDA error";
+    case RCX_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int rcx_rope_freqs(int scheme, double base, int d, int64_t L_train, int64_t L_target, double alpha,
+                   double beta, double* inv_freq_out, double* temperature_out) {
+  return rope_freqs_host(scheme, base, d, L_train, L_target, alpha, beta, inv_freq_out, temperature_out);
+}
+
+int rcx_rope_apply(rcx_tensor q, rcx_tensor k, rcx_tensor q_out, rcx_tensor k_out, const int64_t* positions,
+                   int64_t n_positions, const double* inv_freq, void* stream) {
+  return rope_apply_impl(q, k, q_out, k_out, positions, n_positions, inv_freq, as_stream(stream));
+}
+
+int rcx_attn_blockwise_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                           int64_t kv_block, int64_t window, int64_t n_sink, double temperature, int64_t q_start,
+                           int64_t k_start, const int64_t* positions, int64_t n_positions,
+                           const double* inv_freq, int rope_flags, void* stream) {
+  return attn_impl(q, k, v, o, lse, kv_block, window, n_sink, temperature, q_start, k_start, positions,
+                   n_positions, inv_freq, rope_flags, as_stream(stream));
+}
+
+int rcx_merge_partials(rcx_tensor o_a, rcx_tensor lse_a, rcx_tensor o_b, rcx_tensor lse_b, rcx_tensor o_out,
+                       rcx_tensor lse_out, void* stream) {
+  return merge_impl(o_a, lse_a, o_b, lse_b, o_out, lse_out, as_stream(stream));
+}
+
+int64_t rcx_ring_workspace_size(rcx_tensor q, rcx_tensor k, int64_t kv_block, int rope_flags) {
+  if (check_act(q) || check_act(k) || kv_block < 0) return -1;
+  return ring_plan(q, k, kv_block, rope_flags).total;
+}
+
+int rcx_ring_attn_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse, int64_t kv_block,
+                      int64_t window, int64_t n_sink, double temperature, const int64_t* positions,
+                      int64_t n_positions, const double* inv_freq, int rope_flags, void* workspace,
+                      int64_t workspace_bytes, void* stream) {
+  return ring_impl(q, k, v, o, lse, kv_block, window, n_sink, temperature, positions, n_positions, inv_freq,
+                   rope_flags, workspace, workspace_bytes, as_stream(stream));
+}
+
+int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                           int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+                           const int64_t* positions, int64_t n_positions, const double* inv_freq, int rope_flags,
+                           void* stream) {
+  // Host buffers must be dense [B, N, H, d] / [B, H, N, 1].
+  const rcx_tensor* hs[4] = {&q, &k, &v, &o};
+  for (int i = 0; i < 4; ++i) {
+    const rcx_tensor& t = *hs[i];
+    if (!t.ptr || !shape_ok(t)) return RCX_ERR_INVALID_ARG;
+    if (t.stride[3] != 1 || t.stride[2] != t.shape[3] || t.stride[1] != t.shape[2] * t.shape[3] ||
+        t.stride[0] != t.shape[1] * t.stride[1])
+      return RCX_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  auto bytes = [](const rcx_tensor& t) {
+    return t.shape[0] * t.shape[1] * t.shape[2] * t.shape[3] * (int64_t)elem_size(t.dtype);
+  };
+  const int64_t lse_bytes = lse.ptr ? lse.shape[0] * lse.shape[1] * lse.shape[2] * 4 : 0;
+  const int64_t ws_bytes = rcx_ring_workspace_size(q, k, kv_block, rope_flags);
+  if (ws_bytes < 0) return RCX_ERR_INVALID_ARG;
+  const int64_t pos_bytes = positions ? n_positions * 8 : 0;
+  const int64_t sizes[7] = {bytes(q), bytes(k), bytes(v), bytes(o), lse_bytes, ws_bytes, pos_bytes};
+  int64_t offs[7], total = 0;
+  for (int i = 0; i < 7; ++i) { offs[i] = total; total = align256(total + sizes[i]); }
+  char* dev = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&dev), (size_t)std::max<int64_t>(total, 256), s) != cudaSuccess)
+    return RCX_ERR_CUDA;
+  rcx_tensor dq = q, dk = k, dv = v, dout = o, dl = lse;
+  dq.ptr = dev + offs[0]; dk.ptr = dev + offs[1]; dv.ptr = dev + offs[2]; dout.ptr = dev + offs[3];
+  if (lse.ptr) dl.ptr = dev + offs[4];
+  int64_t* dpos = positions ? reinterpret_cast<int64_t*>(dev + offs[6]) : nullptr;
+  int st = RCX_OK;
+  if (cudaMemcpyAsync(dq.ptr, q.ptr, sizes[0], cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk.ptr, k.ptr, sizes[1], cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv.ptr, v.ptr, sizes[2], cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      (dpos && cudaMemcpyAsync(dpos, positions, pos_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess))
+    st = RCX_ERR_CUDA;
+  if (!st)
+    st = ring_impl(dq, dk, dv, dout, dl, kv_block, window, n_sink, temperature, dpos, n_positions, inv_freq,
+                   rope_flags, dev + offs[5], ws_bytes, s);
+  if (!st && (cudaMemcpyAsync(o.ptr, dout.ptr, sizes[3], cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+              (lse.ptr && cudaMemcpyAsync(lse.ptr, dl.ptr, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)))
+    st = RCX_ERR_CUDA;
+  cudaFreeAsync(dev, s);
+  if (cudaStreamSynchronize(s) != cudaSuccess && !st) st = RCX_ERR_CUDA;
+  return st;
+}
+
+int rcx_device_status(void* stream, int* status_out) {
+  if (!status_out) return RCX_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return RCX_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RCX_ERR_CUDA;
+  *status_out = v;
+  const int zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RCX_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RCX_ERR_CUDA;
+  return RCX_OK;
+}
+
+int rcx_debug_inject_wait_timeout(int64_t spins) {
+  if (spins < 0) return RCX_ERR_INVALID_ARG;
+  attn_tc_set_inject(spins);
+  return RCX_OK;
+}
+
+}  // extern "C"

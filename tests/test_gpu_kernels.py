@@ -1,0 +1,280 @@
+"""GPU parity of each C-ABI call against the float64 oracle (small and ragged
+shapes that span several tiles, plus edge cases).  Calls go through the
+ctypes binding of librcx.so."""
+
+import math
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+from oracle import rcx_oracle as orc
+from rope_context_extension_scaled_b200 import _lib
+from rope_context_extension_scaled_b200.inputs import make_qkv
+from tests._parity import (all_rows, assert_bf16, assert_f32, errors, gather_gpu, np64, oracle_rows)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+# ------------------------------------------------------------------ rope_apply
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N,Hq,Hkv,d", [(37, 3, 1, 64), (300, 8, 2, 128), (1, 1, 1, 128)])
+@pytest.mark.parametrize("pos_kind", ["arange", "random"])
+def test_rope_apply_matches_oracle(dtype, N, Hq, Hkv, d, pos_kind):
+    q, k, _ = make_qkv(2, N, Hq, Hkv, d, dtype, seed=1, device=DEV)
+    inv, _ = _lib.rope_freqs(_lib.NTK, 5e5, d, 8192, 8192 * 128)
+    pos = None
+    p_np = np.arange(N)
+    if pos_kind == "random":
+        g = torch.Generator(device=DEV)
+        g.manual_seed(3)
+        pos = torch.randint(0, 1 << 20, (N,), generator=g, device=DEV, dtype=torch.int64)
+        p_np = pos.cpu().numpy()
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    _lib.rope_apply(q, k, inv, positions=pos, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    for x, y in ((q, qo), (k, ko)):
+        for b in range(2):
+            ref = orc.rope_rotate(np64(x[b]), p_np, inv)
+            got = np64(y[b])
+            if dtype == torch.float32:
+                assert np.abs(got - ref).max() < 1e-5
+            else:   # one bf16 rounding of the fp32 result
+                assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+
+
+def test_rope_apply_in_place_equals_out_of_place():
+    q, k, _ = make_qkv(1, 257, 4, 2, 128, torch.bfloat16, seed=2, device=DEV)
+    inv, _ = _lib.rope_freqs(_lib.YARN, 1e4, 128, 4096, 32768)
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    _lib.rope_apply(q, k, inv, q_out=qo, k_out=ko)
+    q2, k2 = q.clone(), k.clone()
+    _lib.rope_apply(q2, k2, inv)
+    torch.cuda.synchronize()
+    assert torch.equal(q2, qo) and torch.equal(k2, ko)
+    # K only
+    k3 = k.clone()
+    _lib.rope_apply(None, k3, inv)
+    assert torch.equal(k3, ko)
+
+
+def test_rope_angle_error_at_one_million():
+    # Unit vectors (1, 0) in every pair, rotated in fp32: the applied angle
+    # must be within 1e-5 rad of m * theta' (exact, 60-digit arithmetic).
+    d = 128
+    inv, _ = _lib.rope_freqs(_lib.NTK, 5e5, d, 8192, 1 << 20)
+    ms = [0, 1, 65535, 999_999, 1_048_575, (1 << 24) - 1]
+    x = torch.zeros(1, len(ms), 1, d, dtype=torch.float32, device=DEV)
+    x[..., 0::2] = 1.0
+    pos = torch.tensor(ms, dtype=torch.int64, device=DEV)
+    _lib.rope_apply(x, None, inv, positions=pos)
+    out = x[0, :, 0].cpu().numpy().astype(np.float64)
+    got = np.arctan2(out[:, 1::2], out[:, 0::2])
+    mpmath.mp.dps = 60
+    worst = 0.0
+    for r, m in enumerate(ms):
+        for i in range(d // 2):
+            e = mpmath.mpf(m) * mpmath.mpf(float(inv[i]))
+            ex = float(e - 2 * mpmath.pi * mpmath.nint(e / (2 * mpmath.pi)))
+            diff = abs((got[r, i] - ex + math.pi) % (2 * math.pi) - math.pi)
+            worst = max(worst, diff)
+    assert worst <= 1e-5, worst
+    assert worst <= 2e-6, worst      # observed: fp32 sincos of the fp64-reduced angle
+
+
+def test_rope_apply_rejects_misaligned():
+    q = torch.zeros(1, 4, 1, 130, dtype=torch.bfloat16, device=DEV)[..., 1:129]   # 2-byte offset
+    inv, _ = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    with pytest.raises(_lib.RcxError) as e:
+        _lib.rope_apply(q, None, inv)
+    assert e.value.status == _lib.RCX_ERR_ALIGNMENT
+
+
+# ------------------------------------------------------------------ attention
+
+def _run_attn(q, k, v, inv, t, rows=None, **kw):
+    o, lse = _lib.attn_blockwise_fwd(q, k, v, temperature=t, inv_freq=inv, **kw)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+@pytest.mark.parametrize("N,kv_block,window,n_sink", [
+    (512, 64, 0, 0), (200, 0, 0, 0), (333, 50, 40, 3), (97, 7, 0, 0), (130, 0, 16, 0)])
+def test_fp32_attention_fused_rope(N, kv_block, window, n_sink):
+    q, k, v = make_qkv(1, N, 2, 1, 64, torch.float32, seed=4, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.PI, 1e4, 64, 256, 512)
+    o, lse = _run_attn(q, k, v, inv, t, kv_block=kv_block, window=window, n_sink=n_sink,
+                       rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    rows = all_rows(N, 2)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, window, n_sink)
+    assert_f32(errors(*gather_gpu(o, lse, rows), Or, Lr))
+
+
+@pytest.mark.parametrize("N,Hq,Hkv", [(1, 2, 1), (100, 4, 2), (128, 2, 2), (300, 8, 2), (513, 3, 1),
+                                      (640, 4, 4), (257, 6, 3)])
+def test_bf16_tensor_core_attention(N, Hq, Hkv):
+    q, k, v = make_qkv(1, N, Hq, Hkv, 128, torch.bfloat16, seed=5, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 8192, 32768)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    o, lse = _run_attn(q, krot, v, inv, t, rope_flags=_lib.ROTATE_Q)
+    rows = all_rows(N, Hq)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows)
+    assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
+
+
+@pytest.mark.parametrize("window,n_sink,kv_block", [(64, 4, 0), (200, 0, 256), (1000, 2, 0), (129, 130, 384),
+                                                    (0, 0, 384), (0, 0, 100)])
+def test_bf16_window_sinks_ring_order(window, n_sink, kv_block):
+    N = 777
+    q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=6, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.YARN, 1e4, 128, 256, 2048)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    o, lse = _run_attn(q, krot, v, inv, t, rope_flags=_lib.ROTATE_Q, window=window, n_sink=n_sink,
+                       kv_block=kv_block)
+    rows = all_rows(N, 4)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, window, n_sink)
+    assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
+
+
+def test_bf16_offsets_positions_and_fp32_output():
+    # q rows are global tokens 500.., keys 0..; custom positions; fp32 output.
+    Nq, Nk = 200, 700
+    q, _, _ = make_qkv(1, Nq, 4, 2, 128, torch.bfloat16, seed=7, device=DEV)
+    _, k, v = make_qkv(1, Nk, 4, 2, 128, torch.bfloat16, seed=8, device=DEV)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(9)
+    pos = torch.randint(0, 1 << 20, (Nk,), generator=g, device=DEV, dtype=torch.int64)
+    inv, t = _lib.rope_freqs(_lib.DYN_NTK, 5e5, 128, 8192, 131072)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, positions=pos, k_out=krot)
+    o, lse = _run_attn(q, krot, v, inv, t, rope_flags=_lib.ROTATE_Q, q_start=500, k_start=0, positions=pos,
+                       out_dtype=torch.float32)
+    assert o.dtype == torch.float32
+    rows = all_rows(Nq, 4)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, positions=pos, q_start=500, k_start=0)
+    assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_fully_masked_rows_and_empty_inputs(dtype):
+    d = 128 if dtype == torch.bfloat16 else 64
+    q, k, v = make_qkv(1, 64, 2, 1, d, dtype, seed=10, device=DEV)
+    # keys all after the queries: nothing visible
+    o, lse = _lib.attn_blockwise_fwd(q, k, v, q_start=0, k_start=1000)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+    # empty query set is a no-op
+    e = q[:, :0]
+    o2, l2 = _lib.attn_blockwise_fwd(e, k, v)
+    assert o2.shape[1] == 0
+
+
+def test_rotate_k_in_kernel_unsupported_on_tensor_core_path():
+    q, k, v = make_qkv(1, 16, 2, 1, 128, torch.bfloat16, seed=11, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    with pytest.raises(_lib.RcxError) as e:
+        _lib.attn_blockwise_fwd(q, k, v, inv_freq=inv, rope_flags=_lib.ROTATE_K)
+    assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------- merge
+
+@pytest.mark.parametrize("out", ["inplace", "bf16", "f32"])
+def test_merge_partials(out):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(12)
+    B, N, H, d = 2, 77, 3, 128
+    oa = torch.randn(B, N, H, d, generator=g, device=DEV)
+    ob = torch.randn(B, N, H, d, generator=g, device=DEV)
+    la = torch.randn(B, H, N, generator=g, device=DEV) * 5
+    lb = torch.randn(B, H, N, generator=g, device=DEV) * 5
+    la[0, 0, :5] = -math.inf
+    lb[0, 0, 3:8] = -math.inf
+    ro, rl = orc.merge(np64(oa).transpose(0, 2, 1, 3), np64(la), np64(ob).transpose(0, 2, 1, 3), np64(lb))
+    ro = ro.transpose(0, 2, 1, 3)
+    if out == "inplace":
+        oa2, la2 = oa.clone(), la.clone()
+        go, gl = _lib.merge_partials(oa2, la2, ob, lb)
+    else:
+        dt = torch.bfloat16 if out == "bf16" else torch.float32
+        go = torch.empty(B, N, H, d, dtype=dt, device=DEV)
+        gl = torch.empty(B, H, N, device=DEV)
+        _lib.merge_partials(oa, la, ob, lb, go, gl)
+    torch.cuda.synchronize()
+    tol = 1e-5 if out != "bf16" else 2e-2
+    assert np.abs(np64(go) - ro).max() <= tol
+    fin = np.isfinite(rl)
+    assert np.array_equal(np.isneginf(np64(gl)), np.isneginf(rl))
+    assert np.abs(np64(gl)[fin] - rl[fin]).max() <= 1e-5
+
+
+# ----------------------------------------------------------------------- ring
+
+@pytest.mark.parametrize("dtype,d,N,kv_block,window,n_sink", [
+    (torch.bfloat16, 128, 1024, 256, 0, 0), (torch.bfloat16, 128, 1000, 384, 300, 4),
+    (torch.float32, 64, 512, 64, 0, 0), (torch.float32, 64, 300, 128, 50, 2)])
+def test_ring_driver_matches_oracle(dtype, d, N, kv_block, window, n_sink):
+    q, k, v = make_qkv(1, N, 4, 2, d, dtype, seed=13, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.NTK, 1e4, d, 256, 1024)
+    o, lse = _lib.ring_attn_fwd(q, k, v, kv_block=kv_block, window=window, n_sink=n_sink, temperature=t,
+                                inv_freq=inv, rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    torch.cuda.synchronize()
+    rows = all_rows(N, 4)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, window, n_sink)
+    err = errors(*gather_gpu(o, lse, rows), Or, Lr)
+    (assert_bf16 if dtype == torch.bfloat16 else assert_f32)(err)
+
+
+def test_ring_equals_single_call_bf16():
+    N = 1024
+    q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=14, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 256, 2048)
+    o1, l1 = _lib.ring_attn_fwd(q, k, v, kv_block=256, temperature=t, inv_freq=inv,
+                                rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    o2, l2 = _lib.attn_blockwise_fwd(q, krot, v, temperature=t, inv_freq=inv, rope_flags=_lib.ROTATE_Q)
+    torch.cuda.synchronize()
+    # same arithmetic up to the merge points: differences are bf16 output roundings
+    assert (o1.float() - o2.float()).abs().max().item() <= 2 ** -7
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def test_ring_host_buffers_entry_point():
+    N = 512
+    q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=15, device="cpu")
+    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 256, 1024)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(1, 4, N, dtype=torch.float32).pin_memory()
+    _lib.ring_attn_fwd_host(qh, kh, vh, oh, lh, kv_block=128, temperature=t, inv_freq=inv,
+                            rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    od, ld = _lib.ring_attn_fwd(q.cuda(), k.cuda(), v.cuda(), kv_block=128, temperature=t, inv_freq=inv,
+                                rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, od.cpu()) and torch.equal(lh, ld.cpu())
+
+
+# ------------------------------------------------------------ bounded waits
+
+def test_bounded_wait_timeout_reports_and_context_survives():
+    q, k, v = make_qkv(1, 256, 2, 1, 128, torch.bfloat16, seed=16, device=DEV)
+    assert _lib.device_status() == 0
+    _lib.debug_inject_wait_timeout(20000)
+    try:
+        _lib.attn_blockwise_fwd(q, k, v)
+        torch.cuda.synchronize()
+        assert _lib.device_status() == _lib.RCX_ERR_DEVICE_TIMEOUT
+    finally:
+        _lib.debug_inject_wait_timeout(0)
+    # the context still works and the next run is clean
+    o, lse = _lib.attn_blockwise_fwd(q, k, v)
+    torch.cuda.synchronize()
+    assert _lib.device_status() == 0
+    assert torch.isfinite(o.float()).all()
