@@ -213,6 +213,25 @@ int rcx_device_status(void* stream, int* status_out);
  */
 int rcx_debug_inject_wait_timeout(int64_t spins);
 
+/*
+ * Launch accounting, for measurement.  Every kernel launch is counted per
+ * kind.  With timing on, each launch is also bracketed by two CUDA events
+ * recorded on the stream it is launched on; rcx_stats_read() waits for the
+ * last of them and returns the summed elapsed time.  Events are host-side
+ * CUDA objects (no device memory); the pool is kept until process exit.
+ */
+typedef enum {
+    RCX_KERNEL_ROPE = 0,       /* rope_apply                   */
+    RCX_KERNEL_ATTN_TC = 1,    /* tcgen05 bf16 attention       */
+    RCX_KERNEL_ATTN_SIMT = 2,  /* SIMT fp32 attention          */
+    RCX_KERNEL_MERGE = 3,      /* merge_partials               */
+    RCX_KERNEL_KINDS = 4
+} rcx_kernel_kind;
+
+int rcx_stats_enable_timing(int on);
+int rcx_stats_reset(void);
+int rcx_stats_read(int kind, int64_t* launches_out, double* elapsed_ms_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,8 +29,9 @@ EXPORTS = (
     "rcx_abi_version", "rcx_status_string", "rcx_rope_freqs", "rcx_rope_apply",
     "rcx_attn_blockwise_fwd", "rcx_merge_partials", "rcx_ring_workspace_size",
     "rcx_ring_attn_fwd", "rcx_ring_attn_fwd_host", "rcx_device_status",
-    "rcx_debug_inject_wait_timeout",
+    "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
 )
+KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3}
 
 
 class RcxError(RuntimeError):
@@ -72,9 +73,12 @@ def load():
     lib.rcx_ring_attn_fwd_host.argtypes = [T, T, T, T, T, i64, i64, i64, f64, vp, i64, pd, ctypes.c_int, vp]
     lib.rcx_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.rcx_debug_inject_wait_timeout.argtypes = [i64]
+    lib.rcx_stats_enable_timing.argtypes = [ctypes.c_int]
+    lib.rcx_stats_read.argtypes = [ctypes.c_int, ctypes.POINTER(i64), ctypes.POINTER(f64)]
     for name in ("rcx_rope_freqs", "rcx_rope_apply", "rcx_attn_blockwise_fwd", "rcx_merge_partials",
                  "rcx_ring_attn_fwd", "rcx_ring_attn_fwd_host", "rcx_device_status",
-                 "rcx_debug_inject_wait_timeout"):
+                 "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset",
+                 "rcx_stats_read"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -242,3 +246,22 @@ def device_status(device=None):
 
 def debug_inject_wait_timeout(spins):
     _check(load().rcx_debug_inject_wait_timeout(int(spins)), "rcx_debug_inject_wait_timeout")
+
+
+def stats_enable_timing(on=True):
+    _check(load().rcx_stats_enable_timing(1 if on else 0), "rcx_stats_enable_timing")
+
+
+def stats_reset():
+    _check(load().rcx_stats_reset(), "rcx_stats_reset")
+
+
+def stats_read():
+    """{kind: (launches, elapsed_ms)} for every kernel kind."""
+    out = {}
+    for name, k in KERNEL_KINDS.items():
+        n = ctypes.c_int64(0)
+        ms = ctypes.c_double(0.0)
+        _check(load().rcx_stats_read(k, ctypes.byref(n), ctypes.byref(ms)), "rcx_stats_read")
+        out[name] = (n.value, ms.value)
+    return out

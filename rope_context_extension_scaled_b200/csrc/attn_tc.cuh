@@ -710,8 +710,9 @@ static bool tc_view_ok(const rcx_tensor& t) {
   return true;
 }
 
+template <typename ScopeFn>
 static int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v,
-                          const rcx_tensor& o, cudaStream_t stream) {
+                          const rcx_tensor& o, cudaStream_t stream, ScopeFn&& scope_fn) {
   if (!tc_view_ok(q) || !tc_view_ok(k) || !tc_view_ok(v)) return RCX_ERR_ALIGNMENT;
   const int oes = o.dtype == RCX_BF16 ? 2 : 4;
   if (reinterpret_cast<uintptr_t>(o.ptr) % 16 || o.stride[0] % (16 / oes) || o.stride[1] % (16 / oes) ||
@@ -734,6 +735,7 @@ static int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tens
   const int64_t items = (int64_t)p.n_rb * p.n_hg * a.q.B;
   if (items <= 0) return RCX_OK;
   if (items > 0x7fffffff) return RCX_ERR_UNSUPPORTED;
+  auto scope = scope_fn(stream);
   if (o.dtype == RCX_BF16) {
     cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
     attn_tc_kernel<__nv_bfloat16><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);

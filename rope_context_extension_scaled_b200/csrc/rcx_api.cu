@@ -23,6 +23,59 @@ using namespace rcx;
 
 namespace {
 
+// ------------------------------------------------------------ launch accounting
+
+struct Stats {
+  std::mutex mu;
+  bool timing = false;
+  int64_t launches[RCX_KERNEL_KINDS] = {0, 0, 0, 0};
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> spans[RCX_KERNEL_KINDS];
+  std::vector<cudaEvent_t> pool;
+
+  cudaEvent_t take() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+
+Stats& stats() {
+  static Stats* s = new Stats();   // kept until exit
+  return *s;
+}
+
+// Counts a launch of `kind`; with timing on, records events around it.
+class LaunchScope {
+ public:
+  LaunchScope(int kind, cudaStream_t stream) : kind_(kind), stream_(stream) {
+    Stats& st = stats();
+    std::lock_guard<std::mutex> g(st.mu);
+    ++st.launches[kind];
+    if (st.timing) {
+      start_ = st.take();
+      stop_ = st.take();
+      cudaEventRecord(start_, stream_);
+    }
+  }
+  ~LaunchScope() {
+    if (!start_) return;
+    cudaEventRecord(stop_, stream_);
+    Stats& st = stats();
+    std::lock_guard<std::mutex> g(st.mu);
+    st.spans[kind_].push_back({start_, stop_});
+  }
+
+ private:
+  int kind_;
+  cudaStream_t stream_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
+
 constexpr int kAbiVersion = 100;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -164,6 +217,7 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
   const int64_t groups = (a.n_tok + kRopeTok - 1) / kRopeTok;
   const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 8);
+  LaunchScope scope(RCX_KERNEL_ROPE, stream);
   if (dtype == RCX_BF16)
     rope_apply_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, stream>>>(a);
   else
@@ -204,6 +258,7 @@ int merge_impl(const rcx_tensor& oa, const rcx_tensor& la, const rcx_tensor& ob,
   a.d4 = (int)(D / 4);
   const int64_t warps = (a.rows * a.d4 + 31) / 32;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 16));
+  LaunchScope scope(RCX_KERNEL_MERGE, stream);
   if (oo.dtype == RCX_BF16)
     merge_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
   else
@@ -219,6 +274,7 @@ int launch_simt(const AttnArgs& a, cudaStream_t stream) {
   const int64_t tiles = (a.q.N + kSimtBR - 1) / kSimtBR;
   dim3 grid((unsigned)tiles, (unsigned)a.q.H, (unsigned)a.q.B);
   const size_t smem = (size_t)2 * kSimtBC * D * sizeof(float);
+  LaunchScope scope(RCX_KERNEL_ATTN_SIMT, stream);
   if (D == 32) {
     cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attn_simt_kernel<T, Tout, 1><<<grid, kSimtBR * 1, smem, stream>>>(a);
@@ -275,7 +331,7 @@ int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
 
   if (q.dtype == RCX_BF16 && D == 128) {
     if (rope_flags & RCX_ROTATE_K) return RCX_ERR_UNSUPPORTED;
-    return attn_tc_launch(a, q, k, v, o, stream);
+    return attn_tc_launch(a, q, k, v, o, stream, [&](cudaStream_t s) { return LaunchScope(RCX_KERNEL_ATTN_TC, s); });
   }
   if (D != 32 && D != 64 && D != 128) return RCX_ERR_UNSUPPORTED;
   if (q.dtype == RCX_F32)
@@ -511,6 +567,44 @@ int rcx_device_status(void* stream, int* status_out) {
   if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return RCX_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return RCX_ERR_CUDA;
+  return RCX_OK;
+}
+
+int rcx_stats_enable_timing(int on) {
+  Stats& st = stats();
+  std::lock_guard<std::mutex> g(st.mu);
+  st.timing = on != 0;
+  return RCX_OK;
+}
+
+int rcx_stats_reset(void) {
+  Stats& st = stats();
+  std::lock_guard<std::mutex> g(st.mu);
+  for (int k = 0; k < RCX_KERNEL_KINDS; ++k) {
+    st.launches[k] = 0;
+    for (auto& p : st.spans[k]) {
+      cudaEventSynchronize(p.second);
+      st.pool.push_back(p.first);
+      st.pool.push_back(p.second);
+    }
+    st.spans[k].clear();
+  }
+  return RCX_OK;
+}
+
+int rcx_stats_read(int kind, int64_t* launches_out, double* elapsed_ms_out) {
+  if (kind < 0 || kind >= RCX_KERNEL_KINDS) return RCX_ERR_INVALID_ARG;
+  Stats& st = stats();
+  std::lock_guard<std::mutex> g(st.mu);
+  if (launches_out) *launches_out = st.launches[kind];
+  double total = 0.0;
+  for (auto& p : st.spans[kind]) {
+    if (cudaEventSynchronize(p.second) != cudaSuccess) return RCX_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p.first, p.second) != cudaSuccess) return RCX_ERR_CUDA;
+    total += ms;
+  }
+  if (elapsed_ms_out) *elapsed_ms_out = total;
   return RCX_OK;
 }
 
