@@ -43,6 +43,9 @@ WORKLOADS = {
                                       131072, window=4096, n_sink=4, sample_rows=4096),
     "llama3_70b_1m_ring": Workload("llama3_70b_1m_ring", 1, 64, 8, 128, 1 << 20, "bf16", NTK, 5e5, 8192, 1 << 20,
                                    kv_block=65536, ring=True, sample_rows=4096),
+    "llama3_8b_128k_ring": Workload("llama3_8b_128k_ring", 1, 32, 8, 128, 131072, "bf16", NTK, 5e5, 8192, 131072,
+                                    kv_block=32768, ring=True, sample_rows=4096),
 }
 
-ORDER = ["pr1_fp32_512", "llama3_8b_8k", "llama3_70b_32k_yarn", "llama3_8b_128k_window", "llama3_70b_1m_ring"]
+ORDER = ["pr1_fp32_512", "llama3_8b_8k", "llama3_70b_32k_yarn", "llama3_8b_128k_window", "llama3_8b_128k_ring",
+         "llama3_70b_1m_ring"]

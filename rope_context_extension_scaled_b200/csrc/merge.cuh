@@ -48,18 +48,19 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
     const int64_t n = bn % N, b = bn / N;
     float lse = -INFINITY;
     if (valid) {
+      // Issue every load before any arithmetic so they are all in flight.
       const float lsa = a.la[b * a.la_sb + h * a.la_sh + n];
       const float lsb = a.lb[b * a.lb_sb + h * a.lb_sh + n];
+      const float4 x = *reinterpret_cast<const float4*>(
+          reinterpret_cast<const float*>(a.oa.ptr) + b * a.oa.sb + n * a.oa.sn + h * a.oa.sh + 4 * c);
+      const float4 y = *reinterpret_cast<const float4*>(
+          reinterpret_cast<const float*>(a.ob.ptr) + b * a.ob.sb + n * a.ob.sn + h * a.ob.sh + 4 * c);
       const float m = fmaxf(lsa, lsb);
       float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
       if (m != -INFINITY) {
         const float wa = (lsa == -INFINITY) ? 0.f : expf(lsa - m);
         const float wb = (lsb == -INFINITY) ? 0.f : expf(lsb - m);
         const float inv = 1.f / (wa + wb);
-        const float4 x = *reinterpret_cast<const float4*>(
-            reinterpret_cast<const float*>(a.oa.ptr) + b * a.oa.sb + n * a.oa.sn + h * a.oa.sh + 4 * c);
-        const float4 y = *reinterpret_cast<const float4*>(
-            reinterpret_cast<const float*>(a.ob.ptr) + b * a.ob.sb + n * a.ob.sn + h * a.ob.sh + 4 * c);
         const float ca = wa * inv, cb = wb * inv;
         r = make_float4(ca * x.x + cb * y.x, ca * x.y + cb * y.y, ca * x.z + cb * y.z, ca * x.w + cb * y.w);
         lse = m + logf(wa + wb);

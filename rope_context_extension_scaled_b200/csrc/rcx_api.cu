@@ -206,6 +206,29 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   }
   if (positions && n_positions < N) return RCX_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return RCX_OK;
+  const int elems = 16 / elem_size(dtype);
+  const int64_t cph = D / elems;                      // 16-byte chunks per head
+  const int64_t max_chunks = (int64_t)kRopeSlots * kRopeThreads;
+  const int64_t cpt = ((has_q ? q.shape[2] : 0) + (has_k ? k.shape[2] : 0)) * cph;
+  if (cpt > max_chunks) {
+    // More chunks per token than one pass holds: rotate head ranges separately.
+    const int64_t hmax = std::max<int64_t>(1, max_chunks / cph);
+    for (int i = 0; i < 2; ++i) {
+      if (!ins[i]->ptr) continue;
+      for (int64_t h0 = 0; h0 < ins[i]->shape[2]; h0 += hmax) {
+        const int64_t nh = std::min(hmax, ins[i]->shape[2] - h0);
+        rcx_tensor si = *ins[i], so = *outs[i];
+        si.ptr = static_cast<char*>(si.ptr) + h0 * si.stride[2] * elem_size(dtype);
+        so.ptr = static_cast<char*>(so.ptr) + h0 * so.stride[2] * elem_size(dtype);
+        si.shape[2] = so.shape[2] = nh;
+        const rcx_tensor nul = null_tensor();
+        int st = i == 0 ? rope_apply_impl(si, nul, so, nul, positions, n_positions, inv_freq, stream)
+                        : rope_apply_impl(nul, si, nul, so, positions, n_positions, inv_freq, stream);
+        if (st) return st;
+      }
+    }
+    return RCX_OK;
+  }
   RopeArgs a;
   std::memset(&a, 0, sizeof(a));
   if (has_q) { a.q_in = make_view(q); a.q_out = make_view(q_out); }
@@ -214,9 +237,12 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   a.n_tok = B * N;
   a.N = N;
   a.pairs = (int)(D / 2);
+  int64_t tpi = std::min<int64_t>(kRopeMaxTok, std::max<int64_t>(1, max_chunks / cpt));
+  tpi = std::min<int64_t>(tpi, (kRopeMaxTok * 64) / a.pairs);
+  a.tok_per_iter = (int)std::max<int64_t>(1, tpi);
   for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
-  const int64_t groups = (a.n_tok + kRopeTok - 1) / kRopeTok;
-  const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 8);
+  const int64_t groups = (a.n_tok + a.tok_per_iter - 1) / a.tok_per_iter;
+  const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 6);
   LaunchScope scope(RCX_KERNEL_ROPE, stream);
   if (dtype == RCX_BF16)
     rope_apply_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, stream>>>(a);
