@@ -187,6 +187,37 @@ int rcx_ring_attn_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rc
                       int rope_flags, void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
+ * rcx_ring_attn_fwd_noalloc -- rcx_ring_attn_fwd for callers that cannot
+ * allocate device memory, so cannot supply a workspace.  (The source pages
+ * have no counterpart: this exists for deployments, not for the method.)
+ * Typical such callers run inside a framework whose caching allocator owns
+ * the whole device heap, or in a serving loop with a fixed memory budget and
+ * a latency bar that cudaMalloc, which can synchronise the device, would break.
+ *
+ * Same arguments and result as rcx_ring_attn_fwd, minus workspace and
+ * workspace_bytes; the caller still passes q, k, v, o and lse.  The scratch
+ * (fp32 accumulator, one shard's fp32 partial, their LSEs and the rotated K)
+ * lives in a file-scope device array of RCX_NOALLOC_SCRATCH_BYTES that every
+ * GPU which loads this library holds until the process exits.  A request whose
+ * rcx_ring_workspace_size() exceeds that returns RCX_ERR_UNSUPPORTED (with a
+ * message on stderr) before anything is launched.  The call itself makes no
+ * cudaMalloc/cudaFree and calls no allocating library routine.
+ *
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (the device current at that moment) and keeps it;
+ * make that first call on a device before any stream capture.
+ * Every call uses the same array and leaves its last contents there; nothing
+ * in it has to start at zero, because each call writes every scratch byte it
+ * reads.  Calls whose work overlaps on the GPU (different streams, or
+ * different host threads) race on the array: serialise them.
+ */
+#define RCX_NOALLOC_SCRATCH_BYTES (32ll << 20)
+int rcx_ring_attn_fwd_noalloc(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                              int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+                              const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                              int rope_flags, void* stream);
+
+/*
  * Host<->device convenience for callers without device memory management:
  * same as rcx_ring_attn_fwd but q, k, v, o (and lse if non-NULL) are HOST
  * buffers (pinned for full copy speed); the call allocates the device copies

@@ -30,7 +30,9 @@ EXPORTS = (
     "rcx_attn_blockwise_fwd", "rcx_merge_partials", "rcx_ring_workspace_size",
     "rcx_ring_attn_fwd", "rcx_ring_attn_fwd_host", "rcx_device_status",
     "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
+    "rcx_ring_attn_fwd_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 32 << 20   # RCX_NOALLOC_SCRATCH_BYTES in include/rcx.h
 KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3}
 
 
@@ -72,6 +74,8 @@ def load():
     lib.rcx_ring_attn_fwd.argtypes = [T, T, T, T, T, i64, i64, i64, f64, vp, i64, pd, ctypes.c_int, vp, i64, vp]
     lib.rcx_ring_attn_fwd_host.argtypes = [T, T, T, T, T, i64, i64, i64, f64, vp, i64, pd, ctypes.c_int, vp]
     lib.rcx_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.rcx_ring_attn_fwd_noalloc.argtypes = [T, T, T, T, T, i64, i64, i64, f64, vp, i64, pd, ctypes.c_int, vp]
+    lib.rcx_ring_attn_fwd_noalloc.restype = ctypes.c_int
     lib.rcx_debug_inject_wait_timeout.argtypes = [i64]
     lib.rcx_stats_enable_timing.argtypes = [ctypes.c_int]
     lib.rcx_stats_read.argtypes = [ctypes.c_int, ctypes.POINTER(i64), ctypes.POINTER(f64)]
@@ -265,3 +269,17 @@ def stats_read():
         _check(load().rcx_stats_read(k, ctypes.byref(n), ctypes.byref(ms)), "rcx_stats_read")
         out[name] = (n.value, ms.value)
     return out
+
+
+def ring_attn_fwd_noalloc(q, k, v, o, lse=None, kv_block=0, window=0, n_sink=0, temperature=1.0, positions=None,
+                          inv_freq=None, rope_flags=0):
+    """rcx_ring_attn_fwd_noalloc: the ring forward with the library's static
+    scratch instead of a caller workspace, for callers that cannot allocate
+    device memory.  o (and lse) are caller-provided; nothing is allocated."""
+    arr, fp = _freq_ptr(inv_freq)
+    pp, npos = _pos(positions)
+    st = load().rcx_ring_attn_fwd_noalloc(view(q), view(k), view(v), view(o), lse_view(lse), int(kv_block),
+                                          int(window), int(n_sink), float(temperature), pp, npos, fp,
+                                          int(rope_flags), _stream(q.device))
+    _check(st, "rcx_ring_attn_fwd_noalloc")
+    return o, lse

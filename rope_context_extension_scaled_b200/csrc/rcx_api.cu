@@ -581,6 +581,64 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
   return st;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------- ring attention without allocation
+
+// Scratch of rcx_ring_attn_fwd_noalloc: a module-scope device array, so the
+// entry point needs no cudaMalloc.  In host code this name only stands for
+// the array; its device address comes from cudaGetSymbolAddress, once per
+// device, with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RCX_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+int noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RCX_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return RCX_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      std::fprintf(stderr, "librcx: cudaGetSymbolAddress of the no-alloc scratch failed: %s\n",
+                   cudaGetErrorString(e));
+      return RCX_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return RCX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rcx_ring_attn_fwd_noalloc(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                              int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
+                              const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                              int rope_flags, void* stream) {
+  if (check_act(q) || check_act(k) || kv_block < 0) return RCX_ERR_INVALID_ARG;
+  const int64_t need = ring_plan(q, k, kv_block, rope_flags).total;
+  if (need > (int64_t)RCX_NOALLOC_SCRATCH_BYTES) {
+    std::fprintf(stderr,
+                 "librcx: rcx_ring_attn_fwd_noalloc needs %lld bytes of scratch; its static buffer holds %lld\n",
+                 (long long)need, (long long)RCX_NOALLOC_SCRATCH_BYTES);
+    return RCX_ERR_UNSUPPORTED;
+  }
+  void* scratch = nullptr;
+  const int st = noalloc_scratch_address(&scratch);
+  if (st) return st;
+  return ring_impl(q, k, v, o, lse, kv_block, window, n_sink, temperature, positions, n_positions, inv_freq,
+                   rope_flags, scratch, (int64_t)RCX_NOALLOC_SCRATCH_BYTES, as_stream(stream));
+}
+
 int rcx_device_status(void* stream, int* status_out) {
   if (!status_out) return RCX_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
