@@ -232,6 +232,21 @@ def config_dict(w):
     return d
 
 
+def max_over_ranks(x, dist, device="cuda"):
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None or dist.get_world_size() == 1:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world, flops_per_rank_step, ms_per_step):
+    """Whole-job throughput: every rank's useful FLOPs over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def time_steps(run, steps, warmup, stream, dist, world):
     import torch
     for _ in range(warmup):
@@ -249,11 +264,7 @@ def time_steps(run, steps, warmup, stream, dist, world):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if dist is not None and world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist)
     return ms / steps
 
 
@@ -296,7 +307,7 @@ def run_ours(args, w):
         _lib.stats_reset()
         f2 = useful_flops(w2)
         attn_ms2 = st2["attn_tc"][1] / 5
-        secondary = {"workload": w2.name, "value": world * f2 / (ms2 * 1e-3) / 1e12, "unit": "TFLOP/s",
+        secondary = {"workload": w2.name, "value": aggregate_tflops(world, f2, ms2), "unit": "TFLOP/s",
                      "ms_per_step": ms2, "attn_kernel_tflops": f2 / (attn_ms2 * 1e-3) / 1e12,
                      "pct_of_peak": 100.0 * f2 / (ms2 * 1e-3) / 1e12 / peaks["bf16_tflops"],
                      "peak": f"bf16_tflops {peaks['bf16_tflops']} ({peak_src}, burst)",
@@ -311,7 +322,7 @@ def run_ours(args, w):
         ms = time_steps(run, args.steps, args.warmup, stream, dist, world)
     clocks = clk.summary()
     flops = useful_flops(w)
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = aggregate_tflops(world, flops, ms)
 
     # per-kernel time over one more timed pass (CUDA events on the launching stream)
     _lib.stats_reset()
@@ -387,14 +398,10 @@ def run_ours(args, w):
         t0 = time.perf_counter()
         for _ in range(args.e2e_steps):
             host_step()
-        e_ms = (time.perf_counter() - t0) * 1e3 / args.e2e_steps
-        if dist is not None and world > 1:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / args.e2e_steps, dist)
         h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp))
         d2h = op.numel() * op.element_size() + lp.numel() * 4
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+        e2e = {"value": aggregate_tflops(world, flops, e_ms), "unit": "TFLOP/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "api": "rcx_ring_attn_fwd_host (pinned host buffers; copies, device staging and compute)"}
         del qp, kp, vp, op, lp
