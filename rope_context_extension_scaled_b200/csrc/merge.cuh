@@ -31,44 +31,53 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
 
 template <typename Tout>
 __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
-  // d4 divides 32: a warp covers 32 / d4 whole rows per iteration, and the
-  // loop trip count is uniform across the warp, so the in-place LSE write can
-  // wait for every lane's LSE read with __syncwarp().
+  // A warp walks tokens (b, n) and, per token, all heads: 32 / d4 heads per
+  // step, each lane owning 4 consecutive values of one row.  The token index
+  // is divided once per token, not per element.  Loop trip counts are uniform
+  // across the warp, so the in-place LSE write can wait for every lane's LSE
+  // read with __syncwarp().
   const int rows_per_warp = 32 / a.d4;
   const int lane = threadIdx.x & 31;
   const int sub = lane / a.d4, c = lane % a.d4;
   const int64_t H = a.oa.H, N = a.oa.N;
+  const int64_t ntok = a.rows / H;
   const int64_t nwarps = (int64_t)gridDim.x * blockDim.x / 32;
-  for (int64_t rg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; rg * rows_per_warp < a.rows;
-       rg += nwarps) {
-    const int64_t row = rg * rows_per_warp + sub;
-    const bool valid = row < a.rows;
-    const int64_t h = row % H;
-    const int64_t bn = row / H;
-    const int64_t n = bn % N, b = bn / N;
-    float lse = -INFINITY;
-    if (valid) {
-      // Issue every load before any arithmetic so they are all in flight.
-      const float lsa = a.la[b * a.la_sb + h * a.la_sh + n];
-      const float lsb = a.lb[b * a.lb_sb + h * a.lb_sh + n];
-      const float4 x = *reinterpret_cast<const float4*>(
-          reinterpret_cast<const float*>(a.oa.ptr) + b * a.oa.sb + n * a.oa.sn + h * a.oa.sh + 4 * c);
-      const float4 y = *reinterpret_cast<const float4*>(
-          reinterpret_cast<const float*>(a.ob.ptr) + b * a.ob.sb + n * a.ob.sn + h * a.ob.sh + 4 * c);
-      const float m = fmaxf(lsa, lsb);
-      float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (m != -INFINITY) {
-        const float wa = (lsa == -INFINITY) ? 0.f : expf(lsa - m);
-        const float wb = (lsb == -INFINITY) ? 0.f : expf(lsb - m);
-        const float inv = 1.f / (wa + wb);
-        const float ca = wa * inv, cb = wb * inv;
-        r = make_float4(ca * x.x + cb * y.x, ca * x.y + cb * y.y, ca * x.z + cb * y.z, ca * x.w + cb * y.w);
-        lse = m + logf(wa + wb);
+  const float* oa = reinterpret_cast<const float*>(a.oa.ptr);
+  const float* ob = reinterpret_cast<const float*>(a.ob.ptr);
+  Tout* oo = reinterpret_cast<Tout*>(a.oo.ptr);
+  for (int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; tok < ntok; tok += nwarps) {
+    const int64_t b = tok / N, n = tok - b * N;
+    const float* pa = oa + b * a.oa.sb + n * a.oa.sn + 4 * c;
+    const float* pb = ob + b * a.ob.sb + n * a.ob.sn + 4 * c;
+    Tout* po = oo + b * a.oo.sb + n * a.oo.sn + 4 * c;
+    const float* la = a.la + b * a.la_sb + n;
+    const float* lb = a.lb + b * a.lb_sb + n;
+    float* lo = a.lo + b * a.lo_sb + n;
+    for (int64_t h0 = 0; h0 < H; h0 += rows_per_warp) {
+      const int64_t h = h0 + sub;
+      const bool valid = h < H;
+      float lse = -INFINITY;
+      if (valid) {
+        // every load is issued before any arithmetic
+        const float lsa = la[h * a.la_sh];
+        const float lsb = lb[h * a.lb_sh];
+        const float4 x = *reinterpret_cast<const float4*>(pa + h * a.oa.sh);
+        const float4 y = *reinterpret_cast<const float4*>(pb + h * a.ob.sh);
+        const float m = fmaxf(lsa, lsb);
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (m != -INFINITY) {
+          const float wa = (lsa == -INFINITY) ? 0.f : expf(lsa - m);
+          const float wb = (lsb == -INFINITY) ? 0.f : expf(lsb - m);
+          const float inv = 1.f / (wa + wb);
+          const float ca = wa * inv, cb = wb * inv;
+          r = make_float4(ca * x.x + cb * y.x, ca * x.y + cb * y.y, ca * x.z + cb * y.z, ca * x.w + cb * y.w);
+          lse = m + logf(wa + wb);
+        }
+        store4<Tout>(po + h * a.oo.sh, r);
       }
-      store4<Tout>(reinterpret_cast<Tout*>(a.oo.ptr) + b * a.oo.sb + n * a.oo.sn + h * a.oo.sh + 4 * c, r);
+      __syncwarp();
+      if (valid && c == 0) lo[h * a.lo_sh] = lse;
     }
-    __syncwarp();
-    if (valid && c == 0) a.lo[b * a.lo_sb + h * a.lo_sh + n] = lse;
   }
 }
 

@@ -238,7 +238,7 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   a.N = N;
   a.pairs = (int)(D / 2);
   int64_t tpi = std::min<int64_t>(kRopeMaxTok, std::max<int64_t>(1, max_chunks / cpt));
-  tpi = std::min<int64_t>(tpi, (kRopeMaxTok * 64) / a.pairs);
+  tpi = std::min<int64_t>(tpi, kRopeMaxAngles / a.pairs);
   a.tok_per_iter = (int)std::max<int64_t>(1, tpi);
   for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
   const int64_t groups = (a.n_tok + a.tok_per_iter - 1) / a.tok_per_iter;
@@ -282,8 +282,8 @@ int merge_impl(const rcx_tensor& oa, const rcx_tensor& la, const rcx_tensor& ob,
   a.lo_sb = lo.stride[0]; a.lo_sh = lo.stride[1];
   a.rows = B * N * H;
   a.d4 = (int)(D / 4);
-  const int64_t warps = (a.rows * a.d4 + 31) / 32;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 16));
+  const int64_t warps = B * N;     // one warp per token at a time
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8));
   LaunchScope scope(RCX_KERNEL_MERGE, stream);
   if (oo.dtype == RCX_BF16)
     merge_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);

@@ -4,14 +4,14 @@
 // k_n = R(n) W_k x_n with R(m) turning each pair (2i, 2i+1) by m * theta_i.
 //
 // Layout: [B, N, H, d] views, unit stride on d.  A CTA takes T tokens per
-// iteration (T * chunks-per-token ~ 2048 16-byte chunks).  Phase 1 computes the
-// d/2 (cos, sin) pairs of each of the T tokens once into shared memory
-// (float64 angle reduction, see rope_cos_sin) together with each token's
-// row offsets; phase 2 rotates the chunks (8 bf16 or 4 fp32 values) of all Q
-// and K heads of those tokens.  Which (token, head, chunk) a thread handles is
-// the same every iteration, so it is decoded once into registers and no
-// integer division runs in the data loop.  Algorithmic traffic: one read and
-// one write of every element.
+// iteration (T * chunks-per-token ~ 2048 16-byte chunks).  Each iteration
+// first issues the loads of its chunks (8 bf16 or 4 fp32 values; all Q and K
+// heads of the T tokens), then, while they are in flight, computes the d/2
+// (cos, sin) pairs of each token once into shared memory (float64 angle
+// reduction, see rope_cos_sin; two buffers, so one barrier per iteration),
+// then rotates and stores.  Which (token, head, chunk) a thread handles is the
+// same every iteration, so it is decoded once into registers.  Algorithmic
+// traffic: one read and one write of every element.
 #pragma once
 #include "common.cuh"
 
@@ -29,6 +29,7 @@ struct RopeArgs {
 
 constexpr int kRopeThreads = 256;
 constexpr int kRopeMaxTok = 64;
+constexpr int kRopeMaxAngles = 2048;  // T * pairs per buffer
 constexpr int kRopeSlots = 8;       // chunks per thread per iteration (T * chunks/token <= 2048)
 
 template <typename T>
@@ -63,8 +64,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRopeThreads) rope_apply_kernel(const RopeArgs a) {
   constexpr int kElems = 16 / sizeof(T);       // elements per chunk
   constexpr int kPairsPerChunk = kElems / 2;
-  __shared__ float2 cs[kRopeMaxTok * 64];      // T * pairs <= 4096 (host-checked)
-  __shared__ int64_t off[4][kRopeMaxTok];      // per token: q_in, q_out, k_in, k_out row offsets
+  __shared__ float2 cs[2][kRopeMaxAngles];     // T * pairs <= kRopeMaxAngles (host-checked)
   const int pairs = a.pairs;
   const int TPI = a.tok_per_iter;
   const int cph = (2 * pairs) / kElems;        // chunks per head
@@ -87,36 +87,39 @@ __global__ void __launch_bounds__(kRopeThreads) rope_apply_kernel(const RopeArgs
     slot_w[k] = ((isq ? 1u : 0u) << 31) | ((uint32_t)(r / cph) << 16) | (uint32_t)(r % cph);
   }
 
-  for (int64_t tok0 = (int64_t)blockIdx.x * TPI; tok0 < a.n_tok; tok0 += (int64_t)gridDim.x * TPI) {
+  int buf = 0;
+  for (int64_t tok0 = (int64_t)blockIdx.x * TPI; tok0 < a.n_tok; tok0 += (int64_t)gridDim.x * TPI, buf ^= 1) {
     const int ntok = (int)(a.n_tok - tok0 < TPI ? a.n_tok - tok0 : TPI);
-    for (int e = threadIdx.x; e < ntok * pairs; e += blockDim.x) {
-      const int t = e / pairs, i = e - t * pairs;
-      const int64_t tok = tok0 + t;
-      const int64_t b = tok / a.N, n = tok - b * a.N;
-      if (i == 0) {
-        off[0][t] = b * a.q_in.sb + n * a.q_in.sn;
-        off[1][t] = b * a.q_out.sb + n * a.q_out.sn;
-        off[2][t] = b * a.k_in.sb + n * a.k_in.sn;
-        off[3][t] = b * a.k_out.sb + n * a.k_out.sn;
-      }
-      const int64_t m = a.positions ? a.positions[n] : n;
-      float c, s;
-      rope_cos_sin(m, a.f.theta[i], c, s);
-      cs[t * pairs + i] = make_float2(c, s);
-    }
-    __syncthreads();
+    const int64_t b0 = tok0 / a.N, n0 = tok0 - b0 * a.N;
+    // 1. loads of this iteration's chunks
     uint4 u[kRopeSlots];
+    int64_t bo[kRopeSlots], no[kRopeSlots];
 #pragma unroll
     for (int k = 0; k < kRopeSlots; ++k) {
       const int t = slot_t[k];
+      bo[k] = b0;
+      no[k] = n0 + (t < 0 ? 0 : t);
+      while (no[k] >= a.N) { no[k] -= a.N; ++bo[k]; }
       if (t >= 0 && t < ntok) {
         const bool isq = slot_w[k] >> 31;
         const int h = (slot_w[k] >> 16) & 0x7fff, c = slot_w[k] & 0xffff;
         const View4& vi = isq ? a.q_in : a.k_in;
-        const T* src = reinterpret_cast<const T*>(vi.ptr) + off[isq ? 0 : 2][t] + h * vi.sh + c * kElems;
+        const T* src = reinterpret_cast<const T*>(vi.ptr) + bo[k] * vi.sb + no[k] * vi.sn + h * vi.sh + c * kElems;
         u[k] = *reinterpret_cast<const uint4*>(src);
       }
     }
+    // 2. angles of this iteration's tokens (overlaps the loads)
+    for (int e = threadIdx.x; e < ntok * pairs; e += blockDim.x) {
+      const int t = e / pairs, i = e - t * pairs;
+      int64_t n = n0 + t;
+      while (n >= a.N) n -= a.N;
+      const int64_t m = a.positions ? a.positions[n] : n;
+      float c, s;
+      rope_cos_sin(m, a.f.theta[i], c, s);
+      cs[buf][t * pairs + i] = make_float2(c, s);
+    }
+    __syncthreads();
+    // 3. rotate and store
 #pragma unroll
     for (int k = 0; k < kRopeSlots; ++k) {
       const int t = slot_t[k];
@@ -124,12 +127,11 @@ __global__ void __launch_bounds__(kRopeThreads) rope_apply_kernel(const RopeArgs
         const bool isq = slot_w[k] >> 31;
         const int h = (slot_w[k] >> 16) & 0x7fff, c = slot_w[k] & 0xffff;
         const View4& vo = isq ? a.q_out : a.k_out;
-        rope_chunk_regs<T>(u[k], &cs[t * pairs + c * kPairsPerChunk]);
-        T* dst = reinterpret_cast<T*>(vo.ptr) + off[isq ? 1 : 3][t] + h * vo.sh + c * kElems;
+        rope_chunk_regs<T>(u[k], &cs[buf][t * pairs + c * kPairsPerChunk]);
+        T* dst = reinterpret_cast<T*>(vo.ptr) + bo[k] * vo.sb + no[k] * vo.sn + h * vo.sh + c * kElems;
         *reinterpret_cast<uint4*>(dst) = u[k];
       }
     }
-    __syncthreads();
   }
 }
 
