@@ -93,6 +93,19 @@ int rcx_rope_freqs(int scheme, double base, int d, int64_t L_train, int64_t L_ta
                    double alpha, double beta, double* inv_freq_out, double* temperature_out);
 
 /*
+ * rcx_rope_freqs_per_pair -- per-plane rescaled frequencies
+ * theta'_i = base^(-2i/d) / factors[i], i < d/2, in float64 on the host.
+ * "Context window extension: 4K to 1M" 2.5 (LongRoPE): each 2D rotation
+ * plane gets its own scaling factor; plane i interpolates positions by its
+ * factor (m -> m / factors[i]).  The factors come from the caller (the
+ * pages' evolutionary search for them is not part of this library).
+ * d: even, 2..256; factors: HOST array of d/2 positive finite doubles;
+ * inv_freq_out: caller-owned host array of d/2 doubles.
+ * Returns RCX_ERR_INVALID_ARG on a bad argument (output untouched).
+ */
+int rcx_rope_freqs_per_pair(double base, int d, const double* factors, double* inv_freq_out);
+
+/*
  * rcx_rope_apply -- rotate Q and/or K by R(m) ("Context Extension" concept page,
  * Technical principles: each pair of dimensions (2i, 2i+1) turns by
  * phi = m * theta'_i; q_m = R(m) W_q x_m, k_n = R(n) W_k x_n).

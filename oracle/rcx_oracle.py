@@ -149,6 +149,21 @@ def rope_freqs(scheme: int, base: float, d: int, L_train: int, L_target: int,
     return np.asarray(out, dtype=np.float64), float(t)
 
 
+def rope_freqs_per_pair(base: float, d: int, factors) -> np.ndarray:
+    """Per-plane rescaled frequencies theta'_i = theta_i / lambda_i.
+
+    "Context window extension: 4K to 1M" section 2.5 (LongRoPE): instead of
+    one factor for all frequencies, each 2D rotation plane i gets its own
+    scaling factor lambda_i (found by a search that is not part of this
+    path); plane i then interpolates positions by its own factor, m -> m /
+    lambda_i, i.e. theta_i / lambda_i.  Every lambda_i must be positive.
+    """
+    lam = np.asarray(factors, dtype=np.float64)
+    if lam.shape != (d // 2,) or not np.all(np.isfinite(lam)) or not np.all(lam > 0):
+        raise ValueError("need d/2 positive finite factors")
+    return rope_theta(base, d) / lam
+
+
 # --------------------------------------------------------------------------
 # Rotation
 # --------------------------------------------------------------------------

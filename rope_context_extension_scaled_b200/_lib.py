@@ -30,7 +30,7 @@ EXPORTS = (
     "rcx_attn_blockwise_fwd", "rcx_merge_partials", "rcx_ring_workspace_size",
     "rcx_ring_attn_fwd", "rcx_ring_attn_fwd_host", "rcx_device_status",
     "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
-    "rcx_ring_attn_fwd_noalloc",
+    "rcx_ring_attn_fwd_noalloc", "rcx_rope_freqs_per_pair",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20   # RCX_NOALLOC_SCRATCH_BYTES in include/rcx.h
 KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3}
@@ -66,6 +66,8 @@ def load():
     lib.rcx_status_string.argtypes = [ctypes.c_int]
     lib.rcx_rope_freqs.argtypes = [ctypes.c_int, f64, ctypes.c_int, i64, i64, f64, f64, pd, pd]
     lib.rcx_rope_apply.argtypes = [T, T, T, T, vp, i64, pd, vp]
+    lib.rcx_rope_freqs_per_pair.argtypes = [f64, ctypes.c_int, pd, pd]
+    lib.rcx_rope_freqs_per_pair.restype = ctypes.c_int
     lib.rcx_attn_blockwise_fwd.argtypes = [T, T, T, T, T, i64, i64, i64, f64, i64, i64, vp, i64, pd,
                                            ctypes.c_int, vp]
     lib.rcx_merge_partials.argtypes = [T, T, T, T, T, T, vp]
@@ -165,6 +167,18 @@ def rope_freqs(scheme, base, d, L_train, L_target, alpha=1.0, beta=32.0):
                                float(beta), out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)), ctypes.byref(t))
     _check(st, "rcx_rope_freqs")
     return out, t.value
+
+
+def rope_freqs_per_pair(base, d, factors):
+    """theta_i / factors[i] (per-plane rescaling); returns float64 [d/2]."""
+    f = np.ascontiguousarray(np.asarray(factors, dtype=np.float64))
+    if f.shape != (d // 2,):
+        raise ValueError("need d/2 factors")
+    out = np.zeros(d // 2, dtype=np.float64)
+    st = load().rcx_rope_freqs_per_pair(float(base), int(d), f.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                                        out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    _check(st, "rcx_rope_freqs_per_pair")
+    return out
 
 
 def rope_apply(q, k, inv_freq, positions=None, q_out=None, k_out=None):

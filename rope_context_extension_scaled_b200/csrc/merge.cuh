@@ -53,30 +53,50 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
     const float* la = a.la + b * a.la_sb + n;
     const float* lb = a.lb + b * a.lb_sb + n;
     float* lo = a.lo + b * a.lo_sb + n;
-    for (int64_t h0 = 0; h0 < H; h0 += rows_per_warp) {
-      const int64_t h = h0 + sub;
-      const bool valid = h < H;
-      float lse = -INFINITY;
-      if (valid) {
-        // every load is issued before any arithmetic
-        const float lsa = la[h * a.la_sh];
-        const float lsb = lb[h * a.lb_sh];
-        const float4 x = *reinterpret_cast<const float4*>(pa + h * a.oa.sh);
-        const float4 y = *reinterpret_cast<const float4*>(pb + h * a.ob.sh);
-        const float m = fmaxf(lsa, lsb);
-        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (m != -INFINITY) {
-          const float wa = (lsa == -INFINITY) ? 0.f : expf(lsa - m);
-          const float wb = (lsb == -INFINITY) ? 0.f : expf(lsb - m);
-          const float inv = 1.f / (wa + wb);
-          const float ca = wa * inv, cb = wb * inv;
-          r = make_float4(ca * x.x + cb * y.x, ca * x.y + cb * y.y, ca * x.z + cb * y.z, ca * x.w + cb * y.w);
-          lse = m + logf(wa + wb);
+    // Four rows per lane per step: every load of the step is issued before
+    // any arithmetic, so 8 x 16 bytes per lane are in flight.
+    constexpr int kU = 4;
+    for (int64_t h0 = 0; h0 < H; h0 += (int64_t)kU * rows_per_warp) {
+      float lsa[kU], lsb[kU];
+      float4 x[kU], y[kU];
+      bool valid[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t h = h0 + (int64_t)u * rows_per_warp + sub;
+        valid[u] = h < H;
+        if (valid[u]) {
+          lsa[u] = la[h * a.la_sh];
+          lsb[u] = lb[h * a.lb_sh];
+          x[u] = *reinterpret_cast<const float4*>(pa + h * a.oa.sh);
+          y[u] = *reinterpret_cast<const float4*>(pb + h * a.ob.sh);
         }
-        store4<Tout>(po + h * a.oo.sh, r);
+      }
+      float lse[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t h = h0 + (int64_t)u * rows_per_warp + sub;
+        lse[u] = -INFINITY;
+        if (valid[u]) {
+          const float m = fmaxf(lsa[u], lsb[u]);
+          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (m != -INFINITY) {
+            const float wa = (lsa[u] == -INFINITY) ? 0.f : expf(lsa[u] - m);
+            const float wb = (lsb[u] == -INFINITY) ? 0.f : expf(lsb[u] - m);
+            const float inv = 1.f / (wa + wb);
+            const float ca = wa * inv, cb = wb * inv;
+            r = make_float4(ca * x[u].x + cb * y[u].x, ca * x[u].y + cb * y[u].y, ca * x[u].z + cb * y[u].z,
+                            ca * x[u].w + cb * y[u].w);
+            lse[u] = m + logf(wa + wb);
+          }
+          store4<Tout>(po + h * a.oo.sh, r);
+        }
       }
       __syncwarp();
-      if (valid && c == 0) lo[h * a.lo_sh] = lse;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t h = h0 + (int64_t)u * rows_per_warp + sub;
+        if (valid[u] && c == 0) lo[h * a.lo_sh] = lse[u];
+      }
     }
   }
 }

@@ -243,11 +243,16 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
   const int64_t groups = (a.n_tok + a.tok_per_iter - 1) / a.tok_per_iter;
   const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 6);
+  auto same = [](const View4& x, const View4& y) { return x.sb == y.sb && x.sn == y.sn && x.sh == y.sh; };
+  const bool same_layout = (!has_q || same(a.q_in, a.q_out)) && (!has_k || same(a.k_in, a.k_out));
   LaunchScope scope(RCX_KERNEL_ROPE, stream);
-  if (dtype == RCX_BF16)
-    rope_apply_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, stream>>>(a);
-  else
-    rope_apply_kernel<float><<<grid, kRopeThreads, 0, stream>>>(a);
+  if (dtype == RCX_BF16) {
+    if (same_layout) rope_apply_kernel<__nv_bfloat16, true><<<grid, kRopeThreads, 0, stream>>>(a);
+    else rope_apply_kernel<__nv_bfloat16, false><<<grid, kRopeThreads, 0, stream>>>(a);
+  } else {
+    if (same_layout) rope_apply_kernel<float, true><<<grid, kRopeThreads, 0, stream>>>(a);
+    else rope_apply_kernel<float, false><<<grid, kRopeThreads, 0, stream>>>(a);
+  }
   return launch_status();
 }
 
@@ -500,6 +505,10 @@ const char* rcx_status_string(int status) {
 int rcx_rope_freqs(int scheme, double base, int d, int64_t L_train, int64_t L_target, double alpha,
                    double beta, double* inv_freq_out, double* temperature_out) {
   return rope_freqs_host(scheme, base, d, L_train, L_target, alpha, beta, inv_freq_out, temperature_out);
+}
+
+int rcx_rope_freqs_per_pair(double base, int d, const double* factors, double* inv_freq_out) {
+  return rope_freqs_per_pair_host(base, d, factors, inv_freq_out);
 }
 
 int rcx_rope_apply(rcx_tensor q, rcx_tensor k, rcx_tensor q_out, rcx_tensor k_out, const int64_t* positions,

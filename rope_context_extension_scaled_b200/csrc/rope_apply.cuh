@@ -60,8 +60,10 @@ __device__ __forceinline__ void rope_chunk_regs<float>(uint4& u, const float2* c
   u.w = __float_as_uint(x1 * b.y + y1 * b.x);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kRopeThreads) rope_apply_kernel(const RopeArgs a) {
+// kSame: the output views have the input views' strides (in place, or out of
+// place with one layout), so one set of slot offsets serves loads and stores.
+template <typename T, bool kSame>
+__global__ void __launch_bounds__(kRopeThreads, 2) rope_apply_kernel(const RopeArgs a) {
   constexpr int kElems = 16 / sizeof(T);       // elements per chunk
   constexpr int kPairsPerChunk = kElems / 2;
   __shared__ float2 cs[2][kRopeMaxAngles];     // T * pairs <= kRopeMaxAngles (host-checked)
@@ -87,25 +89,42 @@ __global__ void __launch_bounds__(kRopeThreads) rope_apply_kernel(const RopeArgs
     slot_w[k] = ((isq ? 1u : 0u) << 31) | ((uint32_t)(r / cph) << 16) | (uint32_t)(r % cph);
   }
 
+  // Element offsets of this thread's slots relative to the first token of an
+  // iteration: constant while the iteration's tokens stay in one batch entry.
+  int64_t rel_in[kRopeSlots], rel_out[kSame ? 1 : kRopeSlots];
+#pragma unroll
+  for (int k = 0; k < kRopeSlots; ++k) {
+    const bool isq = slot_w[k] >> 31;
+    const int h = (slot_w[k] >> 16) & 0x7fff, c = slot_w[k] & 0xffff;
+    const View4& vi = isq ? a.q_in : a.k_in;
+    const View4& vo = isq ? a.q_out : a.k_out;
+    const int t = slot_t[k] < 0 ? 0 : slot_t[k];
+    rel_in[k] = t * vi.sn + h * vi.sh + c * kElems;
+    if (!kSame) rel_out[kSame ? 0 : k] = t * vo.sn + h * vo.sh + c * kElems;
+  }
+
   int buf = 0;
   for (int64_t tok0 = (int64_t)blockIdx.x * TPI; tok0 < a.n_tok; tok0 += (int64_t)gridDim.x * TPI, buf ^= 1) {
     const int ntok = (int)(a.n_tok - tok0 < TPI ? a.n_tok - tok0 : TPI);
     const int64_t b0 = tok0 / a.N, n0 = tok0 - b0 * a.N;
+    const bool one_batch = n0 + ntok <= a.N;      // no batch boundary inside this iteration
     // 1. loads of this iteration's chunks
     uint4 u[kRopeSlots];
-    int64_t bo[kRopeSlots], no[kRopeSlots];
 #pragma unroll
     for (int k = 0; k < kRopeSlots; ++k) {
       const int t = slot_t[k];
-      bo[k] = b0;
-      no[k] = n0 + (t < 0 ? 0 : t);
-      while (no[k] >= a.N) { no[k] -= a.N; ++bo[k]; }
       if (t >= 0 && t < ntok) {
         const bool isq = slot_w[k] >> 31;
-        const int h = (slot_w[k] >> 16) & 0x7fff, c = slot_w[k] & 0xffff;
         const View4& vi = isq ? a.q_in : a.k_in;
-        const T* src = reinterpret_cast<const T*>(vi.ptr) + bo[k] * vi.sb + no[k] * vi.sn + h * vi.sh + c * kElems;
-        u[k] = *reinterpret_cast<const uint4*>(src);
+        int64_t off;
+        if (one_batch) {
+          off = b0 * vi.sb + n0 * vi.sn + rel_in[k];
+        } else {
+          int64_t bo = b0, no = n0 + t;
+          while (no >= a.N) { no -= a.N; ++bo; }
+          off = bo * vi.sb + no * vi.sn + (rel_in[k] - t * vi.sn);
+        }
+        u[k] = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(vi.ptr) + off);
       }
     }
     // 2. angles of this iteration's tokens (overlaps the loads)
@@ -125,11 +144,19 @@ __global__ void __launch_bounds__(kRopeThreads) rope_apply_kernel(const RopeArgs
       const int t = slot_t[k];
       if (t >= 0 && t < ntok) {
         const bool isq = slot_w[k] >> 31;
-        const int h = (slot_w[k] >> 16) & 0x7fff, c = slot_w[k] & 0xffff;
+        const int c = slot_w[k] & 0xffff;
         const View4& vo = isq ? a.q_out : a.k_out;
+        int64_t off;
+        const int64_t rel = kSame ? rel_in[k] : rel_out[kSame ? 0 : k];
+        if (one_batch) {
+          off = b0 * vo.sb + n0 * vo.sn + rel;
+        } else {
+          int64_t bo = b0, no = n0 + t;
+          while (no >= a.N) { no -= a.N; ++bo; }
+          off = bo * vo.sb + no * vo.sn + (rel - t * vo.sn);
+        }
         rope_chunk_regs<T>(u[k], &cs[buf][t * pairs + c * kPairsPerChunk]);
-        T* dst = reinterpret_cast<T*>(vo.ptr) + bo[k] * vo.sb + no[k] * vo.sn + h * vo.sh + c * kElems;
-        *reinterpret_cast<uint4*>(dst) = u[k];
+        *reinterpret_cast<uint4*>(reinterpret_cast<T*>(vo.ptr) + off) = u[k];
       }
     }
   }

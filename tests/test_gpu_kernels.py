@@ -161,6 +161,22 @@ def test_bf16_offsets_positions_and_fp32_output():
     assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
 
 
+def test_bf16_attention_with_per_plane_factors():
+    # LongRoPE application: an arbitrary per-plane factor vector flows
+    # through K rotation and the fused Q rotation like any other schedule.
+    N = 600
+    q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=17, device=DEV)
+    rng = np.random.default_rng(5)
+    lam = np.exp(rng.uniform(0.0, np.log(32.0), size=64))
+    inv = _lib.rope_freqs_per_pair(5e5, 128, lam)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    o, lse = _run_attn(q, krot, v, inv, 1.0, rope_flags=_lib.ROTATE_Q)
+    rows = all_rows(N, 4)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], orc.rope_freqs_per_pair(5e5, 128, lam), 1.0, rows)
+    assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_fully_masked_rows_and_empty_inputs(dtype):
     d = 128 if dtype == torch.bfloat16 else 64

@@ -33,6 +33,7 @@ MUTATIONS = [
     ("out = theta / s", "out = theta * s"),
     ("s = seq_len / L_train", "s = L_train / seq_len"),
     ("total += min(n_sink, lo)", "total += n_sink"),
+    ("return rope_theta(base, d) / lam", "return rope_theta(base, d) * lam"),
 ]
 
 

@@ -144,6 +144,22 @@ def test_yarn_temperature_closed_forms():
     np.testing.assert_array_equal(f, f2)
 
 
+def test_per_pair_factors_reduce_to_plain_pi_and_ntk_parts():
+    th = orc.rope_theta(1e4, 128)
+    np.testing.assert_array_equal(orc.rope_freqs_per_pair(1e4, 128, np.ones(64)), th)
+    pi, _ = orc.rope_freqs(orc.PI, 1e4, 128, 4096, 4096 * 8)
+    np.testing.assert_allclose(orc.rope_freqs_per_pair(1e4, 128, np.full(64, 8.0)), pi, rtol=1e-15)
+    # NTK-by-parts is a particular factor vector: lambda_i = 1 / f(lambda_i)
+    parts, _ = orc.rope_freqs(orc.NTK_PARTS, 1e4, 128, 4096, 32768)
+    lam = th / parts
+    np.testing.assert_allclose(orc.rope_freqs_per_pair(1e4, 128, lam), parts, rtol=1e-15)
+    assert lam[0] == 1.0 and lam[-1] == 8.0
+    with pytest.raises(ValueError):
+        orc.rope_freqs_per_pair(1e4, 128, np.zeros(64))
+    with pytest.raises(ValueError):
+        orc.rope_freqs_per_pair(1e4, 128, np.ones(63))
+
+
 # ------------------------------------------------------------------- rotation
 
 def test_rotation_quarter_turn_direction():

@@ -46,3 +46,21 @@ def test_rope_freqs_rejects_bad_arguments(bad):
         _lib.rope_freqs(args["scheme"], args["base"], args["d"], args["L_train"], args["L_target"],
                         args["alpha"], args["beta"])
     assert e.value.status == _lib.RCX_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [2, 64, 128, 256])
+def test_per_pair_factors_match_oracle(d):
+    rng = np.random.default_rng(d)
+    lam = np.exp(rng.uniform(0.0, np.log(64.0), size=d // 2))
+    got = _lib.rope_freqs_per_pair(5e5, d, lam)
+    ref = orc.rope_freqs_per_pair(5e5, d, lam)
+    assert np.max(np.abs(got / ref - 1)) < 1e-13
+
+
+@pytest.mark.parametrize("bad", [0.0, -1.0, float("inf"), float("nan")])
+def test_per_pair_factors_reject_bad_values(bad):
+    lam = np.ones(64)
+    lam[7] = bad
+    with pytest.raises(_lib.RcxError) as e:
+        _lib.rope_freqs_per_pair(1e4, 128, lam)
+    assert e.value.status == _lib.RCX_ERR_INVALID_ARG
