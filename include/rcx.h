@@ -163,6 +163,29 @@ int rcx_attn_blockwise_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
                            const double* inv_freq, int rope_flags, void* stream);
 
 /*
+ * rcx_attn_decode_fwd -- attention of one new query token per (batch, head)
+ * against a KV cache ("Context Extension" concept page, KV-cache section:
+ * each generated token computes Q, K, V, appends K, V to the cache and
+ * attends with its Q to the whole cache).  The keys are global tokens
+ * 0 .. Nk-1 as stored (already rotated when they were appended, e.g. with
+ * rcx_rope_apply); the query is global token q_index; mask, GQA, temperature
+ * and LSE as rcx_attn_blockwise_fwd.  The key range is split across CTAs and
+ * the partial results are merged with the LSE rule of rcx_merge_partials.
+ *
+ * q, o: [B, 1, Hq, 128] (q bf16; o bf16 or f32); k, v: [B, Nk, Hkv, 128]
+ * bf16 with Hq / Hkv in {1, 2, 4, 8}; lse: [B, Hq, 1, 1] fp32 or ptr NULL.
+ * rope_flags: RCX_ROTATE_Q (rotate q at positions[q_index]) or 0;
+ * RCX_ROTATE_K returns RCX_ERR_UNSUPPORTED (the cache holds rotated keys).
+ * workspace: device buffer of rcx_attn_decode_workspace_size(q, k) bytes,
+ * 256-byte aligned, caller-owned.  Memory-bound: reads the cache once.
+ */
+int64_t rcx_attn_decode_workspace_size(rcx_tensor q, rcx_tensor k);
+int rcx_attn_decode_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                        int64_t window, int64_t n_sink, double temperature, int64_t q_index,
+                        const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                        int rope_flags, void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
  * rcx_merge_partials -- LSE-weighted merge of two partial results over
  * disjoint key sets: m = max(lse_a, lse_b), w = exp(lse - m),
  * o = (w_a o_a + w_b o_b) / (w_a + w_b), lse = m + ln(w_a + w_b).
@@ -269,7 +292,8 @@ typedef enum {
     RCX_KERNEL_ATTN_TC = 1,    /* tcgen05 bf16 attention       */
     RCX_KERNEL_ATTN_SIMT = 2,  /* SIMT fp32 attention          */
     RCX_KERNEL_MERGE = 3,      /* merge_partials               */
-    RCX_KERNEL_KINDS = 4
+    RCX_KERNEL_DECODE = 4,     /* decode attention + combine   */
+    RCX_KERNEL_KINDS = 5
 } rcx_kernel_kind;
 
 int rcx_stats_enable_timing(int on);

@@ -30,10 +30,11 @@ EXPORTS = (
     "rcx_attn_blockwise_fwd", "rcx_merge_partials", "rcx_ring_workspace_size",
     "rcx_ring_attn_fwd", "rcx_ring_attn_fwd_host", "rcx_device_status",
     "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
-    "rcx_ring_attn_fwd_noalloc", "rcx_rope_freqs_per_pair",
+    "rcx_ring_attn_fwd_noalloc", "rcx_rope_freqs_per_pair", "rcx_attn_decode_workspace_size",
+    "rcx_attn_decode_fwd",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20   # RCX_NOALLOC_SCRATCH_BYTES in include/rcx.h
-KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3}
+KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3, "decode": 4}
 
 
 class RcxError(RuntimeError):
@@ -68,6 +69,10 @@ def load():
     lib.rcx_rope_apply.argtypes = [T, T, T, T, vp, i64, pd, vp]
     lib.rcx_rope_freqs_per_pair.argtypes = [f64, ctypes.c_int, pd, pd]
     lib.rcx_rope_freqs_per_pair.restype = ctypes.c_int
+    lib.rcx_attn_decode_workspace_size.argtypes = [T, T]
+    lib.rcx_attn_decode_workspace_size.restype = i64
+    lib.rcx_attn_decode_fwd.argtypes = [T, T, T, T, T, i64, i64, f64, i64, vp, i64, pd, ctypes.c_int, vp, i64, vp]
+    lib.rcx_attn_decode_fwd.restype = ctypes.c_int
     lib.rcx_attn_blockwise_fwd.argtypes = [T, T, T, T, T, i64, i64, i64, f64, i64, i64, vp, i64, pd,
                                            ctypes.c_int, vp]
     lib.rcx_merge_partials.argtypes = [T, T, T, T, T, T, vp]
@@ -296,4 +301,30 @@ def ring_attn_fwd_noalloc(q, k, v, o, lse=None, kv_block=0, window=0, n_sink=0, 
                                           int(window), int(n_sink), float(temperature), pp, npos, fp,
                                           int(rope_flags), _stream(q.device))
     _check(st, "rcx_ring_attn_fwd_noalloc")
+    return o, lse
+
+
+def attn_decode_fwd(q, k, v, o=None, lse=None, window=0, n_sink=0, temperature=1.0, q_index=None, positions=None,
+                    inv_freq=None, rope_flags=0, workspace=None, want_lse=True):
+    """One query token per (batch, head) against a KV cache k, v [B, Nk, Hkv, 128].
+
+    q: [B, 1, Hq, 128]; q_index defaults to Nk - 1 (the newest cached token)."""
+    B, _, H, D = q.shape
+    if q_index is None:
+        q_index = k.shape[1] - 1
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, 1, dtype=torch.float32, device=q.device)
+    need = load().rcx_attn_decode_workspace_size(view(q), view(k))
+    if need < 0:
+        raise RcxError(RCX_ERR_INVALID_ARG, "rcx_attn_decode_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    arr, fp = _freq_ptr(inv_freq)
+    pp, npos = _pos(positions)
+    st = load().rcx_attn_decode_fwd(view(q), view(k), view(v), view(o), lse_view(lse), int(window), int(n_sink),
+                                    float(temperature), int(q_index), pp, npos, fp, int(rope_flags),
+                                    ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(q.device))
+    _check(st, "rcx_attn_decode_fwd")
     return o, lse

@@ -1,0 +1,250 @@
+// Decode attention over a long KV cache, split over key ranges, bf16, d = 128.
+//
+// "Context Extension" concept page, KV-cache section: each new token computes
+// its Q, K, V, appends K and V to the cache and attends with its Q to the
+// whole cache.  One query row per (batch, head); the keys are global tokens
+// 0 .. Nk-1 (already rotated, as stored in the cache), the query is token
+// q_index, with the causal / window / sink mask of the prefill kernels.
+//
+// Memory-bound: every cached key and value is read once.  A CTA takes one KV
+// head of one batch entry (all G query heads that share it) and one range of
+// keys; its 8 warps split the range.  In a warp, lane l owns dimensions
+// 4l .. 4l+3 and holds those dimensions of all G query rows in registers, so a
+// key row is one coalesced 256-byte read.  The G partial dot products of a
+// key are summed over the warp with a transpose-reduce (each step halves the
+// set of heads a lane carries), after which lane l holds the score of head
+// (l >> (5 - log2 G)).  Keys are taken 16 at a time: batch max, one rescale of
+// the running state, then P V with the per-head p broadcast by shuffles.
+// The 8 warps merge their states in shared memory and the CTA writes an fp32
+// partial (O, LSE); a second kernel merges the partials of all key ranges
+// with the LSE-weighted rule of the ring merge.
+#pragma once
+#include "attn_common.cuh"
+
+namespace rcx {
+
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecBatch = 16;                 // keys per warp step
+constexpr int kDecMaxG = 8;
+
+struct DecodeArgs {
+  View4 q, k, v, o;             // q, o: [B, 1, Hq, 128]; k, v: [B, Nk, Hkv, 128]
+  float* lse;                   // [B, Hq] (stride lse_sb, lse_sh) or null
+  int64_t lse_sb, lse_sh;
+  float* part_o;                // [splits, B, Hq, 128] fp32
+  float* part_lse;              // [splits, B, Hq]
+  int splits;
+  int64_t keys_per_split;
+  int64_t q_index;              // global token index of the query
+  int64_t window, n_sink;
+  float scale_log2;
+  const int64_t* positions;     // nullptr: identity
+  int rope_q;
+  int G;
+  Freqs f;
+};
+
+__device__ __forceinline__ float dec_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const DecodeArgs a) {
+  constexpr int LG = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;   // log2 G
+  const int split = blockIdx.x;
+  const int hk = blockIdx.y;
+  const int64_t b = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int my_head = lane >> (5 - LG);                          // head whose score this lane ends with
+
+  // ---- Q rows of the group in registers (rotated at the query's position)
+  float qv[G][4];
+  const int64_t qpos = a.positions ? a.positions[a.q_index] : a.q_index;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const __nv_bfloat16* qp =
+        reinterpret_cast<const __nv_bfloat16*>(a.q.ptr) + b * a.q.sb + (int64_t)(hk * G + g) * a.q.sh + 4 * lane;
+    const uint2 u = *reinterpret_cast<const uint2*>(qp);
+    const float2 x0 = bf2_to_f2(u.x), x1 = bf2_to_f2(u.y);
+    qv[g][0] = x0.x; qv[g][1] = x0.y; qv[g][2] = x1.x; qv[g][3] = x1.y;
+    if (a.rope_q) {
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        float c, s;
+        rope_cos_sin(qpos, a.f.theta[2 * lane + pp], c, s);
+        const float x = qv[g][2 * pp], y = qv[g][2 * pp + 1];
+        qv[g][2 * pp] = x * c - y * s;
+        qv[g][2 * pp + 1] = x * s + y * c;
+      }
+    }
+  }
+
+  // ---- this warp's key range
+  const int64_t Nk = a.k.N;
+  const int64_t s_lo = (int64_t)split * a.keys_per_split;
+  const int64_t s_hi = min(Nk, s_lo + a.keys_per_split);
+  const int64_t per_warp = (s_hi - s_lo + kDecWarps - 1) / kDecWarps;
+  const int64_t k_lo = s_lo + warp * per_warp;
+  const int64_t k_hi = min(s_hi, k_lo + per_warp);
+  const int64_t qi = a.q_index;
+
+  float m = -INFINITY, l = 0.f;          // state of head my_head (replicated over its lanes)
+  float acc[G][4];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[g][e] = 0.f;
+
+  const __nv_bfloat16* kbase = reinterpret_cast<const __nv_bfloat16*>(a.k.ptr) + b * a.k.sb + hk * a.k.sh + 4 * lane;
+  const __nv_bfloat16* vbase = reinterpret_cast<const __nv_bfloat16*>(a.v.ptr) + b * a.v.sb + hk * a.v.sh + 4 * lane;
+
+  for (int64_t j0 = k_lo; j0 < k_hi; j0 += kDecBatch) {
+    // skip batches with no visible key (window / causal)
+    const int64_t j1 = min(k_hi, j0 + kDecBatch) - 1;
+    if (!tile_any_visible(qi, qi, j0, j1, a.window, a.n_sink)) continue;
+    uint2 kr[kDecBatch], vr[kDecBatch];
+#pragma unroll
+    for (int t = 0; t < kDecBatch; ++t) {
+      const int64_t j = j0 + t;
+      kr[t] = j <= j1 ? *reinterpret_cast<const uint2*>(kbase + j * a.k.sn) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < kDecBatch; ++t) {
+      const int64_t j = j0 + t;
+      vr[t] = j <= j1 ? *reinterpret_cast<const uint2*>(vbase + j * a.v.sn) : make_uint2(0u, 0u);
+    }
+    float sc[kDecBatch];
+#pragma unroll
+    for (int t = 0; t < kDecBatch; ++t) {
+      const float2 k0 = bf2_to_f2(kr[t].x), k1 = bf2_to_f2(kr[t].y);
+      float part[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        part[g] = fmaf(qv[g][3], k1.y, fmaf(qv[g][2], k1.x, fmaf(qv[g][1], k0.y, qv[g][0] * k0.x)));
+      // transpose-reduce: after step o, a lane keeps half of its heads
+#pragma unroll
+      for (int st = 0, n = G; st < LG; ++st, n >>= 1) {
+        const int off = 16 >> st;
+        const bool hi = lane & off;
+#pragma unroll
+        for (int g = 0; g < n / 2; ++g) {
+          const float send = hi ? part[g] : part[g + n / 2];
+          const float keep = hi ? part[g + n / 2] : part[g];
+          part[g] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      float sres = part[0];
+#pragma unroll
+      for (int off = 16 >> LG; off >= 1; off >>= 1) sres += __shfl_xor_sync(0xffffffffu, sres, off);
+      const int64_t j = j0 + t;
+      const bool vis = j <= j1 && mask_visible(qi, j, a.window, a.n_sink);
+      sc[t] = vis ? sres * a.scale_log2 : -INFINITY;
+    }
+    float bm = sc[0];
+#pragma unroll
+    for (int t = 1; t < kDecBatch; ++t) bm = fmaxf(bm, sc[t]);
+    const float m_new = fmaxf(m, bm);
+    const float mref = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = dec_exp2(m - mref);          // 0 when m = -inf
+    float p[kDecBatch];
+    float ps = 0.f;
+#pragma unroll
+    for (int t = 0; t < kDecBatch; ++t) {
+      p[t] = dec_exp2(sc[t] - mref);
+      ps += p[t];
+    }
+    l = l * alpha + ps;
+    m = m_new;
+    // rescale and accumulate every head this lane carries in acc
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float ag = __shfl_sync(0xffffffffu, alpha, g << (5 - LG));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[g][e] *= ag;
+    }
+#pragma unroll
+    for (int t = 0; t < kDecBatch; ++t) {
+      const float2 v0 = bf2_to_f2(vr[t].x), v1 = bf2_to_f2(vr[t].y);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float pg = __shfl_sync(0xffffffffu, p[t], g << (5 - LG));
+        acc[g][0] = fmaf(pg, v0.x, acc[g][0]);
+        acc[g][1] = fmaf(pg, v0.y, acc[g][1]);
+        acc[g][2] = fmaf(pg, v1.x, acc[g][2]);
+        acc[g][3] = fmaf(pg, v1.y, acc[g][3]);
+      }
+    }
+  }
+
+  // ---- merge the warps' states in shared memory
+  __shared__ float sm_m[kDecWarps][kDecMaxG], sm_l[kDecWarps][kDecMaxG];
+  __shared__ float sm_acc[kDecWarps][kDecMaxG][128];
+  if ((lane & ((32 >> LG) - 1)) == 0) {
+    sm_m[warp][my_head] = m;
+    sm_l[warp][my_head] = l;
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sm_acc[warp][g][4 * lane + e] = acc[g][e];
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * 128; e += blockDim.x) {
+    const int g = e / 128, dd = e % 128;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) mm = fmaxf(mm, sm_m[w][g]);
+    const float mr = mm == -INFINITY ? 0.f : mm;
+    float lt = 0.f, ot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+      const float wgt = dec_exp2(sm_m[w][g] - mr);
+      lt += wgt * sm_l[w][g];
+      ot += wgt * sm_acc[w][g][dd];
+    }
+    const int64_t hq = (int64_t)hk * G + g;
+    const int64_t pidx = ((int64_t)split * a.q.B + b) * a.q.H + hq;
+    a.part_o[pidx * 128 + dd] = lt > 0.f ? ot / lt : 0.f;
+    if (dd == 0) a.part_lse[pidx] = lt > 0.f ? (mr + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+  }
+}
+
+// Merge the split partials of one (batch, head) row: thread per 4 dims.
+template <typename Tout>
+__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
+  const int64_t rows = a.q.B * a.q.H;
+  const int64_t total = rows * 32;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = e / 32;
+    const int c = (int)(e % 32);
+    const int64_t b = row / a.q.H, h = row % a.q.H;
+    float mm = -INFINITY;
+    for (int s = 0; s < a.splits; ++s) mm = fmaxf(mm, a.part_lse[(int64_t)s * rows + row]);
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lse = -INFINITY;
+    if (mm != -INFINITY) {
+      float wsum = 0.f;
+      for (int s = 0; s < a.splits; ++s) {
+        const float ls = a.part_lse[(int64_t)s * rows + row];
+        const float w = ls == -INFINITY ? 0.f : expf(ls - mm);
+        const float4 x = *reinterpret_cast<const float4*>(a.part_o + ((int64_t)s * rows + row) * 128 + 4 * c);
+        r.x += w * x.x; r.y += w * x.y; r.z += w * x.z; r.w += w * x.w;
+        wsum += w;
+      }
+      const float inv = 1.f / wsum;
+      r.x *= inv; r.y *= inv; r.z *= inv; r.w *= inv;
+      lse = mm + logf(wsum);
+    }
+    Tout* op = reinterpret_cast<Tout*>(a.o.ptr) + b * a.o.sb + h * a.o.sh + 4 * c;
+    if constexpr (sizeof(Tout) == 2) {
+      *reinterpret_cast<uint2*>(op) = make_uint2(f2_to_bf2(r.x, r.y), f2_to_bf2(r.z, r.w));
+    } else {
+      *reinterpret_cast<float4*>(op) = r;
+    }
+    if (c == 0 && a.lse) a.lse[b * a.lse_sb + h * a.lse_sh] = lse;
+  }
+}
+
+}  // namespace rcx

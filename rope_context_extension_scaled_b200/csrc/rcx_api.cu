@@ -17,6 +17,7 @@
 #include "attn_common.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_decode.cuh"
 #include "rope_freqs.inc"
 
 using namespace rcx;
@@ -28,7 +29,7 @@ namespace {
 struct Stats {
   std::mutex mu;
   bool timing = false;
-  int64_t launches[RCX_KERNEL_KINDS] = {0, 0, 0, 0};
+  int64_t launches[RCX_KERNEL_KINDS] = {0, 0, 0, 0, 0};
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> spans[RCX_KERNEL_KINDS];
   std::vector<cudaEvent_t> pool;
 
@@ -81,6 +82,8 @@ constexpr int kAbiVersion = 100;
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 inline int elem_size(int dtype) { return dtype == RCX_BF16 ? 2 : 4; }
+
+int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
 bool shape_ok(const rcx_tensor& t) {
   for (int i = 0; i < 4; ++i)
@@ -206,6 +209,54 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   }
   if (positions && n_positions < N) return RCX_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return RCX_OK;
+  {
+    // Dense views (every token one contiguous row, in and out) take the
+    // bulk-copy kernel, one launch per operand.
+    auto dense = [](const rcx_tensor& t) {
+      return t.stride[3] == 1 && t.stride[2] == t.shape[3] && t.stride[1] == t.shape[2] * t.shape[3] &&
+             (t.shape[0] == 1 || t.stride[0] == t.shape[1] * t.stride[1]);
+    };
+    bool all_dense = true;
+    for (int i = 0; i < 2; ++i)
+      if (ins[i]->ptr) {
+        const int64_t tb = ins[i]->shape[2] * D * elem_size(dtype);
+        all_dense = all_dense && dense(*ins[i]) && dense(*outs[i]) && tb <= kRopeBulkBytes && tb % 16 == 0;
+      }
+    if (all_dense) {
+      const size_t smem = (size_t)kRopeBulkStages * kRopeBulkBytes + kRopeMaxAngles * sizeof(float2) +
+                          kRopeBulkStages * sizeof(uint64_t);
+      for (int i = 0; i < 2; ++i) {
+        if (!ins[i]->ptr) continue;
+        RopeBulkArgs b;
+        std::memset(&b, 0, sizeof(b));
+        b.in = ins[i]->ptr;
+        b.out = outs[i]->ptr;
+        b.positions = positions;
+        b.n_tok = B * N;
+        b.N = N;
+        b.d = (int)D;
+        b.pairs = (int)(D / 2);
+        b.token_bytes = ins[i]->shape[2] * D * elem_size(dtype);
+        b.tok_per_chunk = (int)std::max<int64_t>(
+            1, std::min<int64_t>(kRopeBulkBytes / b.token_bytes, kRopeMaxAngles / b.pairs));
+        for (int j = 0; j < b.pairs; ++j) b.f.theta[j] = inv_freq[j];
+        const int64_t chunks = (b.n_tok + b.tok_per_chunk - 1) / b.tok_per_chunk;
+        const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 2);
+        LaunchScope scope(RCX_KERNEL_ROPE, stream);
+        if (dtype == RCX_BF16) {
+          cudaFuncSetAttribute(rope_bulk_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+          rope_bulk_kernel<__nv_bfloat16><<<grid, kRopeThreads, smem, stream>>>(b);
+        } else {
+          cudaFuncSetAttribute(rope_bulk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+          rope_bulk_kernel<float><<<grid, kRopeThreads, smem, stream>>>(b);
+        }
+        const int st = launch_status();
+        if (st) return st;
+      }
+      return RCX_OK;
+    }
+  }
   const int elems = 16 / elem_size(dtype);
   const int64_t cph = D / elems;                      // 16-byte chunks per head
   const int64_t max_chunks = (int64_t)kRopeSlots * kRopeThreads;
@@ -371,6 +422,98 @@ int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
                             : launch_simt<__nv_bfloat16, __nv_bfloat16>(a, stream);
 }
 
+// --------------------------------------------------------------------- decode
+
+struct DecodePlan {
+  int splits;
+  int64_t keys_per_split, off_lse, total;
+};
+
+DecodePlan decode_plan(const rcx_tensor& q, const rcx_tensor& k) {
+  DecodePlan p;
+  const int64_t B = q.shape[0], Hq = q.shape[2], Nk = k.shape[1], Hkv = std::max<int64_t>(k.shape[2], 1);
+  const int64_t want = std::max<int64_t>(1, (2 * (int64_t)sm_count() + Hkv * B - 1) / std::max<int64_t>(1, Hkv * B));
+  const int64_t cap = std::max<int64_t>(1, (Nk + 127) / 128);
+  p.splits = (int)std::min<int64_t>(std::min<int64_t>(want, cap), 4096);
+  p.keys_per_split = std::max<int64_t>(1, (Nk + p.splits - 1) / p.splits);
+  p.off_lse = align256((int64_t)p.splits * B * Hq * 128 * 4);
+  p.total = align256(p.off_lse + (int64_t)p.splits * B * Hq * 4);
+  return p;
+}
+
+int decode_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, const rcx_tensor& o,
+                const rcx_tensor& lse, int64_t window, int64_t n_sink, double temperature, int64_t q_index,
+                const int64_t* positions, int64_t n_positions, const double* inv_freq, int rope_flags,
+                void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
+  int st;
+  if ((st = check_act(q)) || (st = check_act(k)) || (st = check_act(v)) || (st = check_act(o))) return st;
+  const int64_t B = q.shape[0], Hq = q.shape[2], D = q.shape[3], Nk = k.shape[1], Hkv = k.shape[2];
+  if (q.shape[1] != 1 || o.shape[1] != 1) return RCX_ERR_INVALID_ARG;
+  if (q.dtype != RCX_BF16 || k.dtype != RCX_BF16 || v.dtype != RCX_BF16) return RCX_ERR_UNSUPPORTED;
+  if (D != 128 || k.shape[3] != 128 || v.shape[3] != 128 || o.shape[3] != 128) return RCX_ERR_UNSUPPORTED;
+  if (k.shape[0] != B || v.shape[0] != B || o.shape[0] != B || v.shape[1] != Nk || v.shape[2] != Hkv ||
+      o.shape[2] != Hq)
+    return RCX_ERR_INVALID_ARG;
+  if (Hkv <= 0 || Hq % Hkv) return RCX_ERR_INVALID_ARG;
+  const int64_t G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return RCX_ERR_UNSUPPORTED;
+  if (lse.ptr && (st = check_lse(lse, B, Hq, 1))) return st;
+  if (window < 0 || n_sink < 0 || q_index < 0) return RCX_ERR_INVALID_ARG;
+  if (!(temperature > 0.0) || !std::isfinite(temperature)) return RCX_ERR_INVALID_ARG;
+  if (rope_flags & ~RCX_ROTATE_Q) return rope_flags & RCX_ROTATE_K ? RCX_ERR_UNSUPPORTED : RCX_ERR_INVALID_ARG;
+  if (rope_flags && !inv_freq) return RCX_ERR_INVALID_ARG;
+  if (positions && n_positions <= std::max(q_index, Nk - 1)) return RCX_ERR_INVALID_ARG;
+  // 8-byte row accesses for q, k, v; 16 (fp32) or 8 (bf16) for o
+  auto al = [](const rcx_tensor& t, int bytes) {
+    const int per = bytes / elem_size(t.dtype);
+    return reinterpret_cast<uintptr_t>(t.ptr) % bytes == 0 && t.stride[0] % per == 0 && t.stride[1] % per == 0 &&
+           t.stride[2] % per == 0;
+  };
+  if (!al(q, 8) || !al(k, 8) || !al(v, 8) || !al(o, o.dtype == RCX_BF16 ? 8 : 16)) return RCX_ERR_ALIGNMENT;
+  if (B == 0 || Hq == 0) return RCX_OK;
+  if (B > 65535 || Hkv > 65535) return RCX_ERR_UNSUPPORTED;
+  const DecodePlan p = decode_plan(q, k);
+  if (!workspace || workspace_bytes < p.total) return RCX_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return RCX_ERR_ALIGNMENT;
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = make_view(q); a.k = make_view(k); a.v = make_view(v); a.o = make_view(o);
+  a.lse = static_cast<float*>(lse.ptr);
+  a.lse_sb = lse.ptr ? lse.stride[0] : 0;
+  a.lse_sh = lse.ptr ? lse.stride[1] : 0;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.off_lse);
+  a.splits = p.splits;
+  a.keys_per_split = p.keys_per_split;
+  a.q_index = q_index;
+  a.window = window; a.n_sink = n_sink;
+  a.scale_log2 = (float)(1.4426950408889634074 / (std::sqrt((double)D) * temperature));
+  a.positions = positions;
+  a.rope_q = rope_flags & RCX_ROTATE_Q;
+  a.G = (int)G;
+  if (a.rope_q)
+    for (int i = 0; i < 64; ++i) a.f.theta[i] = inv_freq[i];
+  {
+    dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
+    LaunchScope scope(RCX_KERNEL_DECODE, stream);
+    switch (G) {
+      case 1: attn_decode_kernel<1><<<grid, kDecThreads, 0, stream>>>(a); break;
+      case 2: attn_decode_kernel<2><<<grid, kDecThreads, 0, stream>>>(a); break;
+      case 4: attn_decode_kernel<4><<<grid, kDecThreads, 0, stream>>>(a); break;
+      default: attn_decode_kernel<8><<<grid, kDecThreads, 0, stream>>>(a); break;
+    }
+    if ((st = launch_status())) return st;
+  }
+  const int64_t threads = B * Hq * 32;
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 8));
+  LaunchScope scope(RCX_KERNEL_DECODE, stream);
+  if (o.dtype == RCX_BF16)
+    decode_combine_kernel<__nv_bfloat16><<<grid2, 256, 0, stream>>>(a);
+  else
+    decode_combine_kernel<float><<<grid2, 256, 0, stream>>>(a);
+  return launch_status();
+}
+
 // ----------------------------------------------------------------------- ring
 
 struct RingPlan {
@@ -378,8 +521,6 @@ struct RingPlan {
   bool rotate_k_separately;
   int64_t off_acc, off_lacc, off_part, off_lpart, off_krot, total;
 };
-
-int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
 RingPlan ring_plan(const rcx_tensor& q, const rcx_tensor& k, int64_t kv_block, int rope_flags) {
   RingPlan p;
@@ -522,6 +663,19 @@ int rcx_attn_blockwise_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
                            const double* inv_freq, int rope_flags, void* stream) {
   return attn_impl(q, k, v, o, lse, kv_block, window, n_sink, temperature, q_start, k_start, positions,
                    n_positions, inv_freq, rope_flags, as_stream(stream));
+}
+
+int64_t rcx_attn_decode_workspace_size(rcx_tensor q, rcx_tensor k) {
+  if (check_act(q) || check_act(k)) return -1;
+  return decode_plan(q, k).total;
+}
+
+int rcx_attn_decode_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse, int64_t window,
+                        int64_t n_sink, double temperature, int64_t q_index, const int64_t* positions,
+                        int64_t n_positions, const double* inv_freq, int rope_flags, void* workspace,
+                        int64_t workspace_bytes, void* stream) {
+  return decode_impl(q, k, v, o, lse, window, n_sink, temperature, q_index, positions, n_positions, inv_freq,
+                     rope_flags, workspace, workspace_bytes, as_stream(stream));
 }
 
 int rcx_merge_partials(rcx_tensor o_a, rcx_tensor lse_a, rcx_tensor o_b, rcx_tensor lse_b, rcx_tensor o_out,

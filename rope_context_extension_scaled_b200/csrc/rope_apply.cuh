@@ -162,4 +162,156 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_apply_kernel(const RopeA
   }
 }
 
+// ---------------------------------------------------------------------------
+// Bulk-copy path for dense layouts ([B, N, H, d] with no gaps, in and out).
+// A token's H x d values are one contiguous row, so a chunk of T tokens is one
+// contiguous span: cp.async.bulk brings it into shared memory (four stages per
+// CTA, three loading while one is rotated; two CTAs per SM), the CTA computes
+// the chunk's T x d/2 (cos, sin) pairs once, and rotates the span on its way
+// out with coalesced 16-byte stores.  Every wait on a copy is bounded (about
+// one second) and
+// records RCX_ERR_DEVICE_TIMEOUT if it runs out.
+
+constexpr int kRopeBulkStages = 4;
+constexpr int kRopeBulkBytes = 18432;      // bytes of one stage (T * token bytes)
+
+struct RopeBulkArgs {
+  const void* in;
+  void* out;
+  const int64_t* positions;    // nullptr: m = n
+  int64_t n_tok;               // B * N
+  int64_t N;
+  int64_t token_bytes;         // H * d * element size
+  int tok_per_chunk;           // T
+  int pairs;                   // d / 2
+  int d;
+  Freqs f;
+};
+
+__device__ __forceinline__ uint32_t rb_smem(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool rb_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok = 0;
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (it == 0) t0 = t;
+    else if (t - t0 > 1000000000ull) {
+      record_device_error(RCX_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBulkArgs a) {
+  constexpr int kElems = 16 / sizeof(T);
+  constexpr int kPairsPerChunk = kElems / 2;
+  extern __shared__ __align__(128) uint8_t rb_raw[];
+  uint8_t* stage_buf = rb_raw;                                                   // [stages][kRopeBulkBytes]
+  float2* cs = reinterpret_cast<float2*>(rb_raw + kRopeBulkStages * kRopeBulkBytes);   // [T * pairs]
+  uint64_t* full = reinterpret_cast<uint64_t*>(cs + kRopeMaxAngles);             // [stages]
+  __shared__ int abort_flag;
+
+  const int64_t n_chunks = (a.n_tok + a.tok_per_chunk - 1) / a.tok_per_chunk;
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  auto chunk_tokens = [&](int64_t c) {
+    const int64_t t0 = c * a.tok_per_chunk;
+    const int64_t left = a.n_tok - t0;
+    return (int)(left < a.tok_per_chunk ? left : a.tok_per_chunk);
+  };
+  auto issue_load = [&](int64_t c, int st) {
+    const int64_t t0 = c * a.tok_per_chunk;
+    const uint32_t bytes = (uint32_t)(chunk_tokens(c) * a.token_bytes);
+    const uint32_t bar = rb_smem(&full[st]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            rb_smem(stage_buf + st * kRopeBulkBytes)),
+        "l"(static_cast<const uint8_t*>(a.in) + t0 * a.token_bytes), "r"(bytes), "r"(bar)
+        : "memory");
+  };
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int st = 0; st < kRopeBulkStages; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(rb_smem(&full[st])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int st = 0; st < kRopeBulkStages; ++st)
+      if (first + st * step < n_chunks) issue_load(first + st * step, st);
+  }
+  __syncthreads();
+
+  int i = 0;
+  for (int64_t c = first; c < n_chunks; c += step, ++i) {
+    const int st = i % kRopeBulkStages;
+    const int ntok = chunk_tokens(c);
+    const int64_t t0 = c * a.tok_per_chunk;
+    // angles of the chunk's tokens (while the copy lands)
+    const int64_t n0 = t0 - (t0 / a.N) * a.N;
+    for (int e = threadIdx.x; e < ntok * a.pairs; e += blockDim.x) {
+      const int t = e / a.pairs, p = e - t * a.pairs;
+      int64_t n = n0 + t;
+      while (n >= a.N) n -= a.N;
+      const int64_t m = a.positions ? a.positions[n] : n;
+      float cc, sn;
+      rope_cos_sin(m, a.f.theta[p], cc, sn);
+      cs[t * a.pairs + p] = make_float2(cc, sn);
+    }
+    if (threadIdx.x == 0 && !rb_wait(rb_smem(&full[st]), (i / kRopeBulkStages) & 1)) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    // rotate the span out of shared memory into global memory (plain
+    // coalesced 16-byte stores: nothing waits for them, so the stage is free
+    // as soon as every thread has read it)
+    const uint8_t* buf = stage_buf + st * kRopeBulkBytes;
+    uint8_t* dst = static_cast<uint8_t*>(a.out) + t0 * a.token_bytes;
+    const int row_chunks = (int)(a.token_bytes / 16);
+    const int d_chunks = a.d / kElems;
+    for (int e = threadIdx.x; e < ntok * row_chunks; e += blockDim.x) {
+      const int t = e / row_chunks, rc = e - t * row_chunks;
+      const int dc = rc % d_chunks;                      // 16-byte chunk within the head
+      uint4 u = *reinterpret_cast<const uint4*>(buf + (size_t)e * 16);
+      rope_chunk_regs<T>(u, &cs[t * a.pairs + dc * kPairsPerChunk]);
+      *reinterpret_cast<uint4*>(dst + (size_t)e * 16) = u;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const int64_t nc = c + (int64_t)kRopeBulkStages * step;
+      if (nc < n_chunks) issue_load(nc, st);
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (abort_flag) {
+      // let copies that may still be landing finish before the CTA exits
+      for (int st = 0; st < kRopeBulkStages; ++st) {
+        uint32_t ok;
+        uint64_t t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        do {
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+              "selp.u32 %0, 1, 0, p;\n\t}"
+              : "=r"(ok)
+              : "r"(rb_smem(&full[st])), "r"(0u)
+              : "memory");
+          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        } while (!ok && t - t0 < 100000000ull);
+      }
+    }
+  }
+}
+
 }  // namespace rcx

@@ -294,3 +294,43 @@ def test_bounded_wait_timeout_reports_and_context_survives():
     torch.cuda.synchronize()
     assert _lib.device_status() == 0
     assert torch.isfinite(o.float()).all()
+
+
+# --------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("B,Nk,Hq,Hkv,window,n_sink,qoff", [
+    (1, 1, 1, 1, 0, 0, 0), (2, 1000, 8, 1, 0, 0, 0), (1, 5000, 8, 8, 0, 0, 0), (2, 3333, 16, 4, 0, 0, 0),
+    (1, 20000, 64, 8, 4096, 4, 0), (1, 777, 4, 2, 100, 3, 0), (1, 4096, 8, 2, 0, 0, 50)])
+def test_decode_split_kv_matches_oracle(B, Nk, Hq, Hkv, window, n_sink, qoff):
+    qf, _, _ = make_qkv(B, 1, Hq, Hkv, 128, torch.bfloat16, seed=20, device=DEV)
+    _, k, v = make_qkv(B, Nk, Hq, Hkv, 128, torch.bfloat16, seed=21, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 8192, 131072)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)                 # the cache holds rotated keys
+    q_index = Nk - 1 + qoff                                    # newest token (or later: all keys visible)
+    pos = None
+    if qoff:
+        pos = torch.arange(q_index + 1, dtype=torch.int64, device=DEV)
+    o, lse = _lib.attn_decode_fwd(qf, krot, v, window=window, n_sink=n_sink, temperature=t, q_index=q_index,
+                                  positions=pos, inv_freq=inv, rope_flags=_lib.ROTATE_Q)
+    torch.cuda.synchronize()
+    for b in range(B):
+        rows = {h: np.array([0]) for h in range(Hq)}
+        Or, Lr = oracle_rows(qf[b], k[b], v[b], inv, t, rows, window, n_sink, q_start=q_index, k_start=0)
+        Og = {h: np64(o[b, 0, h, :])[None] for h in range(Hq)}
+        Lg = {h: np.array([float(lse[b, h, 0])]) for h in range(Hq)}
+        err = errors(Og, Lg, Or, Lr)
+        assert err["inf_ok"] and err["o_max"] <= 2e-2 and err["lse_max"] <= 1e-3, err
+
+
+def test_decode_rejects_rotate_k_and_bad_group():
+    q, k, v = make_qkv(1, 1, 6, 2, 128, torch.bfloat16, seed=22, device=DEV)   # G = 3
+    _, kc, vc = make_qkv(1, 64, 6, 2, 128, torch.bfloat16, seed=23, device=DEV)
+    with pytest.raises(_lib.RcxError) as e:
+        _lib.attn_decode_fwd(q, kc, vc)
+    assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
+    q2, _, _ = make_qkv(1, 1, 4, 2, 128, torch.bfloat16, seed=24, device=DEV)
+    inv, _ = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    with pytest.raises(_lib.RcxError) as e:
+        _lib.attn_decode_fwd(q2, kc, vc, inv_freq=inv, rope_flags=_lib.ROTATE_K)
+    assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
