@@ -360,6 +360,26 @@ def run_ours(args, w):
         kern["merge"] = {"launches_per_step": st["merge"][0] / reps, "ms_per_step": m_ms,
                          "gbs": m_bytes / (m_ms * 1e-3) / 1e9 if m_ms else None,
                          "pct_hbm": 100 * m_bytes / (m_ms * 1e-3) / 1e9 / peaks["hbm_gbs"] if m_ms else None}
+    # ---------------- decode: one new query token per head against the same KV cache
+    decode = None
+    if args.decode and w.dtype == "bf16":
+        qd = q[:, -1:].contiguous()
+        od = torch.empty_like(qd)
+        ld = torch.empty(w.B, w.Hq, 1, dtype=torch.float32, device="cuda")
+        inv_d, t_d = _lib.rope_freqs(w.scheme, w.base, w.d, w.L_train, w.L_target, w.alpha, w.beta)
+        wsd = torch.empty(max(_lib.load().rcx_attn_decode_workspace_size(_lib.view(qd), _lib.view(k)), 256),
+                          dtype=torch.uint8, device="cuda")
+
+        def dstep():
+            _lib.attn_decode_fwd(qd, k, v, od, ld, window=w.window, n_sink=w.n_sink, temperature=t_d,
+                                 q_index=w.N - 1, inv_freq=inv_d, rope_flags=_lib.ROTATE_Q, workspace=wsd)
+        d_ms = time_steps(dstep, 20, 5, stream, dist, world)
+        kv_bytes = 2.0 * k.numel() * k.element_size()
+        decode = {"workload": f"decode: 1 query token per head, {w.N}-token KV cache, {w.Hq}/{w.Hkv} heads",
+                  "ms": d_ms, "gbs": kv_bytes / (d_ms * 1e-3) / 1e9,
+                  "pct_hbm": 100.0 * kv_bytes / (d_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                  "tokens_per_s": world * w.B / (d_ms * 1e-3)}
+        del qd, od, ld, wsd
     peak_key = "bf16_tflops_sustained" if ms > 1000 else "bf16_tflops"
     peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
     achieved = flops / (attn_ms * 1e-3) / 1e12
@@ -429,7 +449,7 @@ def run_ours(args, w):
             "pct_of_peak": 100.0 * value / world / peak, "peak": f"{peak_key} {peak} ({peak_src})",
             "tokens_per_s": world * w.B * w.N / (ms * 1e-3),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches * args.steps),
-            "kernels": kern, "clocks": clocks, "secondary": secondary}
+            "kernels": kern, "clocks": clocks, "secondary": secondary, "decode": decode}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -450,6 +470,7 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=1)
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
+    ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture (reported as roofline.traffic)")
     args = ap.parse_args()
