@@ -167,8 +167,9 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_apply_kernel(const RopeA
 // A token's H x d values are one contiguous row, so a chunk of T tokens is one
 // contiguous span: cp.async.bulk brings it into shared memory (four stages per
 // CTA, three loading while one is rotated; two CTAs per SM), the CTA computes
-// the chunk's T x d/2 (cos, sin) pairs once, and rotates the span on its way
-// out with coalesced 16-byte stores.  Every wait on a copy is bounded (about
+// the chunk's T x d/2 (cos, sin) pairs once (with consecutive positions: one
+// precise angle per pair and the angle-addition identity for the rest), and
+// rotates the span on its way out with coalesced 16-byte stores.  Every wait on a copy is bounded (about
 // one second) and
 // records RCX_ERR_DEVICE_TIMEOUT if it runs out.
 
@@ -260,14 +261,33 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBu
     const int64_t t0 = c * a.tok_per_chunk;
     // angles of the chunk's tokens (while the copy lands)
     const int64_t n0 = t0 - (t0 / a.N) * a.N;
-    for (int e = threadIdx.x; e < ntok * a.pairs; e += blockDim.x) {
-      const int t = e / a.pairs, p = e - t * a.pairs;
-      int64_t n = n0 + t;
-      while (n >= a.N) n -= a.N;
-      const int64_t m = a.positions ? a.positions[n] : n;
-      float cc, sn;
-      rope_cos_sin(m, a.f.theta[p], cc, sn);
-      cs[t * a.pairs + p] = make_float2(cc, sn);
+    if (!a.positions && n0 + ntok <= a.N) {
+      // Consecutive positions n0, n0 + 1, ...: the first angle of each pair
+      // precisely, the next ones by the angle-addition identity
+      // (cos, sin)((m + 1) theta) = (cos, sin)(m theta) * (cos, sin)(theta);
+      // at most T - 1 complex products, ~1 ulp each.
+      for (int p = threadIdx.x; p < a.pairs; p += blockDim.x) {
+        float cc, sn, c1, s1;
+        rope_cos_sin(n0, a.f.theta[p], cc, sn);
+        rope_cos_sin(1, a.f.theta[p], c1, s1);
+        cs[p] = make_float2(cc, sn);
+        for (int t = 1; t < ntok; ++t) {
+          const float c2 = cc * c1 - sn * s1, s2 = sn * c1 + cc * s1;
+          cc = c2;
+          sn = s2;
+          cs[t * a.pairs + p] = make_float2(cc, sn);
+        }
+      }
+    } else {
+      for (int e = threadIdx.x; e < ntok * a.pairs; e += blockDim.x) {
+        const int t = e / a.pairs, p = e - t * a.pairs;
+        int64_t n = n0 + t;
+        while (n >= a.N) n -= a.N;
+        const int64_t m = a.positions ? a.positions[n] : n;
+        float cc, sn;
+        rope_cos_sin(m, a.f.theta[p], cc, sn);
+        cs[t * a.pairs + p] = make_float2(cc, sn);
+      }
     }
     if (threadIdx.x == 0 && !rb_wait(rb_smem(&full[st]), (i / kRopeBulkStages) & 1)) abort_flag = 1;
     __syncthreads();
