@@ -336,12 +336,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- work item: (row block, head group, batch), heaviest row blocks first
+  // ---- work item: (batch, KV head, row block, head group within the KV
+  // head), KV head slowest so that the CTAs resident at any time stream the
+  // same K/V block (which then stays in L2), heaviest row blocks first.
   const int item = blockIdx.x;
-  const int per_rb = P.n_hg * (int)a.q.B;
-  const int rb = P.n_rb - 1 - item / per_rb;
-  const int hg = (item % per_rb) % P.n_hg;
-  const int64_t bb = (item % per_rb) / P.n_hg;
+  const int hg_per_kv = P.n_hg / (int)a.k.H;
+  const int per_kv = P.n_rb * hg_per_kv;
+  const int per_b = per_kv * (int)a.k.H;
+  const int64_t bb = item / per_b;
+  const int kv_i = (item % per_b) / per_kv;
+  const int rem = (item % per_b) % per_kv;
+  const int rb = P.n_rb - 1 - rem / hg_per_kv;
+  const int hg = kv_i * hg_per_kv + rem % hg_per_kv;
   int head[2];
   int64_t row0[2];
   if (P.pair_heads) {
