@@ -36,6 +36,11 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "causal attention fwd TFLOP/s and % of B200 BF16 tensor peak at 128K and 1M"
+# DRAM bytes (read + write) per attention launch, from a one-pass ncu capture of
+# every attention launch of one step of the same command (summary and command in
+# profiles/attn_tc_traffic_llama3_70b_1m_ring.md).  Valid for the attention
+# kernel as captured; re-take it when the kernel changes.
+ATTN_TRAFFIC_PER_LAUNCH = {"llama3_70b_1m_ring": 3.743e9}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -383,8 +388,9 @@ def run_ours(args, w):
     peak_key = "bf16_tflops_sustained" if ms > 1000 else "bf16_tflops"
     peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
     achieved = flops / (attn_ms * 1e-3) / 1e12
+    traffic = args.traffic if args.traffic is not None else ATTN_TRAFFIC_PER_LAUNCH.get(w.name)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": args.traffic, "kernel": attn_key,
+                "traffic": traffic, "kernel": attn_key,
                 "peak_source": f"{peak_key} ({peak_src})"}
     del run
     torch.cuda.empty_cache()
