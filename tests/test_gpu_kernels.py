@@ -334,3 +334,56 @@ def test_decode_rejects_rotate_k_and_bad_group():
     with pytest.raises(_lib.RcxError) as e:
         _lib.attn_decode_fwd(q2, kc, vc, inv_freq=inv, rope_flags=_lib.ROTATE_K)
     assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------ batch > 1, G = 8
+
+def _oracle_batch(q, k, v, inv, t, window=0, n_sink=0):
+    out = []
+    for b in range(q.shape[0]):
+        rows = all_rows(q.shape[1], q.shape[2])
+        out.append((rows, *oracle_rows(q[b], k[b], v[b], inv, t, rows, window, n_sink)))
+    return out
+
+
+@pytest.mark.parametrize("Hq,Hkv,window,n_sink", [(16, 2, 0, 0), (8, 1, 300, 4), (6, 2, 0, 0)])
+def test_bf16_tensor_core_batch2(Hq, Hkv, window, n_sink):
+    B, N = 2, 700
+    q, k, v = make_qkv(B, N, Hq, Hkv, 128, torch.bfloat16, seed=30, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.YARN, 1e4, 128, 512, 4096)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    o, lse = _lib.attn_blockwise_fwd(q, krot, v, temperature=t, inv_freq=inv, rope_flags=_lib.ROTATE_Q,
+                                     window=window, n_sink=n_sink)
+    torch.cuda.synchronize()
+    for b, (rows, Or, Lr) in enumerate(_oracle_batch(q, k, v, inv, t, window, n_sink)):
+        Og = {h: np64(o[b, r, h, :]) for h, r in rows.items()}
+        Lg = {h: lse[b, h, r].cpu().numpy().astype(np.float64) for h, r in rows.items()}
+        assert_bf16(errors(Og, Lg, Or, Lr))
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_ring_batch2(dtype, d):
+    B, N = 2, 640
+    q, k, v = make_qkv(B, N, 8, 2, d, dtype, seed=31, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, d, 256, 2048)
+    o, lse = _lib.ring_attn_fwd(q, k, v, kv_block=256, temperature=t, inv_freq=inv,
+                                rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    torch.cuda.synchronize()
+    for b, (rows, Or, Lr) in enumerate(_oracle_batch(q, k, v, inv, t)):
+        Og = {h: np64(o[b, r, h, :]) for h, r in rows.items()}
+        Lg = {h: lse[b, h, r].cpu().numpy().astype(np.float64) for h, r in rows.items()}
+        (assert_bf16 if dtype == torch.bfloat16 else assert_f32)(errors(Og, Lg, Or, Lr))
+
+
+def test_rope_apply_batch_wrap_in_chunk():
+    # N smaller than a bulk chunk: chunks straddle batch entries (direct angles).
+    B, N = 5, 3
+    q, k, _ = make_qkv(B, N, 2, 8, 128, torch.bfloat16, seed=32, device=DEV)
+    inv, _ = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    ko = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=ko)
+    torch.cuda.synchronize()
+    for b in range(B):
+        ref = orc.rope_rotate(np64(k[b]), np.arange(N), inv)
+        assert np.all(np.abs(np64(ko[b]) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
