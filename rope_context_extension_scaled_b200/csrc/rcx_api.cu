@@ -238,7 +238,7 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
         b.pairs = (int)(D / 2);
         b.token_bytes = ins[i]->shape[2] * D * elem_size(dtype);
         b.tok_per_chunk = (int)std::max<int64_t>(
-            1, std::min<int64_t>(kRopeBulkBytes / b.token_bytes, kRopeMaxAngles / b.pairs));
+            1, std::min<int64_t>(kRopeBulkBytes / b.token_bytes, (kRopeMaxAngles / 2) / b.pairs));
         for (int j = 0; j < b.pairs; ++j) b.f.theta[j] = inv_freq[j];
         const int64_t chunks = (b.n_tok + b.tok_per_chunk - 1) / b.tok_per_chunk;
         const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 2);

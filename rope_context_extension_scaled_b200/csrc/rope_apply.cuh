@@ -166,10 +166,11 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_apply_kernel(const RopeA
 // Bulk-copy path for dense layouts ([B, N, H, d] with no gaps, in and out).
 // A token's H x d values are one contiguous row, so a chunk of T tokens is one
 // contiguous span: cp.async.bulk brings it into shared memory (four stages per
-// CTA, three loading while one is rotated; two CTAs per SM), the CTA computes
-// the chunk's T x d/2 (cos, sin) pairs once (with consecutive positions: one
-// precise angle per pair and the angle-addition identity for the rest), and
-// rotates the span on its way out with coalesced 16-byte stores.  Every wait on a copy is bounded (about
+// CTA, three loading while one is rotated; two CTAs per SM).  Two warps build
+// the next chunk's T x d/2 (cos, sin) table (with consecutive positions: one
+// precise angle per pair and the angle-addition identity for the rest) while
+// six warps rotate the current chunk on its way out with coalesced 16-byte
+// stores.  Every wait on a copy is bounded (about
 // one second) and
 // records RCX_ERR_DEVICE_TIMEOUT if it runs out.
 
@@ -217,19 +218,23 @@ __device__ __forceinline__ bool rb_wait(uint32_t bar, uint32_t parity) {
 
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBulkArgs a) {
+  // Warps 0-5 rotate chunk i while warps 6-7 build the angle table of chunk
+  // i + 1 into the other table buffer; one barrier per chunk.
   constexpr int kElems = 16 / sizeof(T);
   constexpr int kPairsPerChunk = kElems / 2;
+  constexpr int kRotThreads = kRopeThreads - 64;
   extern __shared__ __align__(128) uint8_t rb_raw[];
-  uint8_t* stage_buf = rb_raw;                                                   // [stages][kRopeBulkBytes]
-  float2* cs = reinterpret_cast<float2*>(rb_raw + kRopeBulkStages * kRopeBulkBytes);   // [T * pairs]
-  uint64_t* full = reinterpret_cast<uint64_t*>(cs + kRopeMaxAngles);             // [stages]
+  uint8_t* stage_buf = rb_raw;                                                        // [stages][kRopeBulkBytes]
+  float2* cs = reinterpret_cast<float2*>(rb_raw + kRopeBulkStages * kRopeBulkBytes);  // [2][kRopeMaxAngles / 2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(cs + kRopeMaxAngles);                  // [stages]
   __shared__ int abort_flag;
+  constexpr int kTab = kRopeMaxAngles / 2;
 
   const int64_t n_chunks = (a.n_tok + a.tok_per_chunk - 1) / a.tok_per_chunk;
   const int64_t first = blockIdx.x, step = gridDim.x;
+  const bool rot = threadIdx.x < kRotThreads;
   auto chunk_tokens = [&](int64_t c) {
-    const int64_t t0 = c * a.tok_per_chunk;
-    const int64_t left = a.n_tok - t0;
+    const int64_t left = a.n_tok - c * a.tok_per_chunk;
     return (int)(left < a.tok_per_chunk ? left : a.tok_per_chunk);
   };
   auto issue_load = [&](int64_t c, int st) {
@@ -243,6 +248,39 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBu
         "l"(static_cast<const uint8_t*>(a.in) + t0 * a.token_bytes), "r"(bytes), "r"(bar)
         : "memory");
   };
+  // Angle table of chunk c into cs[buf]: one precise angle per pair and the
+  // angle-addition identity for consecutive positions, else direct angles.
+  auto build_table = [&](int64_t c, int buf) {
+    const int lt = threadIdx.x - kRotThreads;          // 0 .. 63
+    const int ntok = chunk_tokens(c);
+    const int64_t t0 = c * a.tok_per_chunk;
+    const int64_t n0 = t0 - (t0 / a.N) * a.N;
+    float2* tab = cs + buf * kTab;
+    if (!a.positions && n0 + ntok <= a.N) {
+      for (int p = lt; p < a.pairs; p += 64) {
+        float cc, sn, c1, s1;
+        rope_cos_sin(n0, a.f.theta[p], cc, sn);
+        rope_cos_sin(1, a.f.theta[p], c1, s1);
+        tab[p] = make_float2(cc, sn);
+        for (int t = 1; t < ntok; ++t) {
+          const float c2 = cc * c1 - sn * s1, s2 = sn * c1 + cc * s1;
+          cc = c2;
+          sn = s2;
+          tab[t * a.pairs + p] = make_float2(cc, sn);
+        }
+      }
+    } else {
+      for (int e = lt; e < ntok * a.pairs; e += 64) {
+        const int t = e / a.pairs, p = e - t * a.pairs;
+        int64_t n = n0 + t;
+        while (n >= a.N) n -= a.N;
+        const int64_t m = a.positions ? a.positions[n] : n;
+        float cc, sn;
+        rope_cos_sin(m, a.f.theta[p], cc, sn);
+        tab[t * a.pairs + p] = make_float2(cc, sn);
+      }
+    }
+  };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -252,84 +290,57 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBu
     for (int st = 0; st < kRopeBulkStages; ++st)
       if (first + st * step < n_chunks) issue_load(first + st * step, st);
   }
+  if (!rot && first < n_chunks) build_table(first, 0);
   __syncthreads();
 
   int i = 0;
   for (int64_t c = first; c < n_chunks; c += step, ++i) {
     const int st = i % kRopeBulkStages;
-    const int ntok = chunk_tokens(c);
-    const int64_t t0 = c * a.tok_per_chunk;
-    // angles of the chunk's tokens (while the copy lands)
-    const int64_t n0 = t0 - (t0 / a.N) * a.N;
-    if (!a.positions && n0 + ntok <= a.N) {
-      // Consecutive positions n0, n0 + 1, ...: the first angle of each pair
-      // precisely, the next ones by the angle-addition identity
-      // (cos, sin)((m + 1) theta) = (cos, sin)(m theta) * (cos, sin)(theta);
-      // at most T - 1 complex products, ~1 ulp each.
-      for (int p = threadIdx.x; p < a.pairs; p += blockDim.x) {
-        float cc, sn, c1, s1;
-        rope_cos_sin(n0, a.f.theta[p], cc, sn);
-        rope_cos_sin(1, a.f.theta[p], c1, s1);
-        cs[p] = make_float2(cc, sn);
-        for (int t = 1; t < ntok; ++t) {
-          const float c2 = cc * c1 - sn * s1, s2 = sn * c1 + cc * s1;
-          cc = c2;
-          sn = s2;
-          cs[t * a.pairs + p] = make_float2(cc, sn);
+    const int buf = i & 1;
+    if (rot) {
+      if (!rb_wait(rb_smem(&full[st]), (i / kRopeBulkStages) & 1)) abort_flag = 1;
+      if (!abort_flag) {
+        const int ntok = chunk_tokens(c);
+        const int64_t t0 = c * a.tok_per_chunk;
+        const uint8_t* src = stage_buf + st * kRopeBulkBytes;
+        uint8_t* dst = static_cast<uint8_t*>(a.out) + t0 * a.token_bytes;
+        const float2* tab = cs + buf * kTab;
+        const int row_chunks = (int)(a.token_bytes / 16);
+        const int d_chunks = a.d / kElems;
+        for (int e = threadIdx.x; e < ntok * row_chunks; e += kRotThreads) {
+          const int t = e / row_chunks, rc = e - t * row_chunks;
+          const int dc = rc % d_chunks;                  // 16-byte chunk within the head
+          uint4 u = *reinterpret_cast<const uint4*>(src + (size_t)e * 16);
+          rope_chunk_regs<T>(u, &tab[t * a.pairs + dc * kPairsPerChunk]);
+          *reinterpret_cast<uint4*>(dst + (size_t)e * 16) = u;
         }
       }
-    } else {
-      for (int e = threadIdx.x; e < ntok * a.pairs; e += blockDim.x) {
-        const int t = e / a.pairs, p = e - t * a.pairs;
-        int64_t n = n0 + t;
-        while (n >= a.N) n -= a.N;
-        const int64_t m = a.positions ? a.positions[n] : n;
-        float cc, sn;
-        rope_cos_sin(m, a.f.theta[p], cc, sn);
-        cs[t * a.pairs + p] = make_float2(cc, sn);
-      }
+    } else if (c + step < n_chunks) {
+      build_table(c + step, buf ^ 1);
     }
-    if (threadIdx.x == 0 && !rb_wait(rb_smem(&full[st]), (i / kRopeBulkStages) & 1)) abort_flag = 1;
     __syncthreads();
     if (abort_flag) break;
-    // rotate the span out of shared memory into global memory (plain
-    // coalesced 16-byte stores: nothing waits for them, so the stage is free
-    // as soon as every thread has read it)
-    const uint8_t* buf = stage_buf + st * kRopeBulkBytes;
-    uint8_t* dst = static_cast<uint8_t*>(a.out) + t0 * a.token_bytes;
-    const int row_chunks = (int)(a.token_bytes / 16);
-    const int d_chunks = a.d / kElems;
-    for (int e = threadIdx.x; e < ntok * row_chunks; e += blockDim.x) {
-      const int t = e / row_chunks, rc = e - t * row_chunks;
-      const int dc = rc % d_chunks;                      // 16-byte chunk within the head
-      uint4 u = *reinterpret_cast<const uint4*>(buf + (size_t)e * 16);
-      rope_chunk_regs<T>(u, &cs[t * a.pairs + dc * kPairsPerChunk]);
-      *reinterpret_cast<uint4*>(dst + (size_t)e * 16) = u;
-    }
-    __syncthreads();
     if (threadIdx.x == 0) {
       const int64_t nc = c + (int64_t)kRopeBulkStages * step;
       if (nc < n_chunks) issue_load(nc, st);
     }
   }
-  if (threadIdx.x == 0) {
-    if (abort_flag) {
-      // let copies that may still be landing finish before the CTA exits
-      for (int st = 0; st < kRopeBulkStages; ++st) {
-        uint32_t ok;
-        uint64_t t0, t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-        do {
-          asm volatile(
-              "{\n\t.reg .pred p;\n\t"
-              "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-              "selp.u32 %0, 1, 0, p;\n\t}"
-              : "=r"(ok)
-              : "r"(rb_smem(&full[st])), "r"(0u)
-              : "memory");
-          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        } while (!ok && t - t0 < 100000000ull);
-      }
+  if (threadIdx.x == 0 && abort_flag) {
+    // let copies that may still be landing finish before the CTA exits
+    for (int st = 0; st < kRopeBulkStages; ++st) {
+      uint32_t ok;
+      uint64_t t0, t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+      do {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(rb_smem(&full[st])), "r"(0u)
+            : "memory");
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      } while (!ok && t - t0 < 100000000ull);
     }
   }
 }
