@@ -112,7 +112,9 @@ int rcx_rope_freqs_per_pair(double base, int d, const double* factors, double* i
  *
  * q, k: [B, N, H, d] inputs (bf16 or f32); q_out, k_out: outputs of the same
  * shape and dtype (out.ptr == in.ptr rotates in place; an operand whose
- * in.ptr is NULL is skipped).  positions: device int64 array of n_positions
+ * in.ptr is NULL is skipped).  d <= 256 and a multiple of 8 (bf16) or 4
+ * (f32); base pointers 16-byte aligned and strides multiples of 16 bytes, else
+ * RCX_ERR_ALIGNMENT.  positions: device int64 array of n_positions
  * >= N entries, position of token n is positions[n]; NULL means m = n.
  * inv_freq: HOST array of d/2 doubles (from rcx_rope_freqs).
  * Angles are reduced modulo 2 pi in float64 before an fp32 sincos, so the
@@ -149,10 +151,11 @@ int rcx_rope_apply(rcx_tensor q, rcx_tensor k, rcx_tensor q_out, rcx_tensor k_ou
  * n_positions entries; NULL = identity).  rope_flags == 0: Q and K are taken
  * as already rotated.
  *
- * Paths: f32 inputs run a SIMT fp32 kernel (any d <= 128, even).  bf16 inputs
- * with d == 128 run the tcgen05/TMEM tensor-core kernel; it rotates Q in its
- * tile load and needs K pre-rotated (RCX_ROTATE_K returns
- * RCX_ERR_UNSUPPORTED there: rotate K once with rcx_rope_apply).
+ * Paths: bf16 inputs with d == 128 run the tcgen05/TMEM tensor-core kernel;
+ * it rotates Q in its tile load and needs K pre-rotated (RCX_ROTATE_K returns
+ * RCX_ERR_UNSUPPORTED there: rotate K once with rcx_rope_apply).  Other
+ * inputs (f32, or bf16 with d != 128) run a SIMT fp32-arithmetic kernel for
+ * d in {32, 64, 128}; other d return RCX_ERR_UNSUPPORTED.
  * Alignment: bf16 tensor-core path needs 16-byte aligned base pointers and
  * token/head strides that are multiples of 8 elements.
  */

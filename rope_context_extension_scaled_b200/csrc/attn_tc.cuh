@@ -28,6 +28,7 @@
 // TMA copies and MMAs drain, frees TMEM and returns.
 #pragma once
 #include <cudaTypedefs.h>
+#include <atomic>
 #include "attn_common.cuh"
 
 namespace rcx {
@@ -673,18 +674,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-static int64_t g_tc_inject_spins = 0;
-inline void attn_tc_set_inject(int64_t spins) { g_tc_inject_spins = spins; }
+static std::atomic<int64_t> g_tc_inject_spins{0};
+inline void attn_tc_set_inject(int64_t spins) { g_tc_inject_spins.store(spins); }
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // looked up once, thread-safely
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
 }
 
@@ -737,18 +739,21 @@ static int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tens
   const int64_t rows_per_item = p.pair_heads ? kTcBM : 2 * kTcBM;
   p.n_rb = (int)((a.q.N + rows_per_item - 1) / rows_per_item);
   p.n_hg = (int)(p.pair_heads ? a.q.H / 2 : a.q.H);
-  p.inject_spins = g_tc_inject_spins;
+  p.inject_spins = g_tc_inject_spins.load();
   const int64_t items = (int64_t)p.n_rb * p.n_hg * a.q.B;
   if (items <= 0) return RCX_OK;
   if (items > 0x7fffffff) return RCX_ERR_UNSUPPORTED;
+  const cudaError_t ea = o.dtype == RCX_BF16
+                             ? cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal)
+                             : cudaFuncSetAttribute(attn_tc_kernel<float>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+  if (ea != cudaSuccess) return RCX_ERR_CUDA;
   auto scope = scope_fn(stream);
-  if (o.dtype == RCX_BF16) {
-    cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+  if (o.dtype == RCX_BF16)
     attn_tc_kernel<__nv_bfloat16><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
-  } else {
-    cudaFuncSetAttribute(attn_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
+  else
     attn_tc_kernel<float><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
-  }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RCX_OK : RCX_ERR_CUDA;
 }

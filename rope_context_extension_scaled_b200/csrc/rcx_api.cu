@@ -122,14 +122,23 @@ int check_lse(const rcx_tensor& t, int64_t B, int64_t H, int64_t N) {
 }
 
 int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
+  // initialised once, thread-safely (every device this library targets is a B200)
+  static const int n = [] {
+    int dev = 0, c = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+      c = 148;
+    return c;
+  }();
   return n;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory.
+template <typename K>
+int allow_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
+             ? RCX_OK
+             : RCX_ERR_CUDA;
 }
 
 int launch_status() {
@@ -244,11 +253,10 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
         const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 2);
         LaunchScope scope(RCX_KERNEL_ROPE, stream);
         if (dtype == RCX_BF16) {
-          cudaFuncSetAttribute(rope_bulk_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+          if (allow_smem(rope_bulk_kernel<__nv_bfloat16>, smem)) return RCX_ERR_CUDA;
           rope_bulk_kernel<__nv_bfloat16><<<grid, kRopeThreads, smem, stream>>>(b);
         } else {
-          cudaFuncSetAttribute(rope_bulk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+          if (allow_smem(rope_bulk_kernel<float>, smem)) return RCX_ERR_CUDA;
           rope_bulk_kernel<float><<<grid, kRopeThreads, smem, stream>>>(b);
         }
         const int st = launch_status();
@@ -358,13 +366,13 @@ int launch_simt(const AttnArgs& a, cudaStream_t stream) {
   const size_t smem = (size_t)2 * kSimtBC * D * sizeof(float);
   LaunchScope scope(RCX_KERNEL_ATTN_SIMT, stream);
   if (D == 32) {
-    cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (allow_smem(attn_simt_kernel<T, Tout, 1>, smem)) return RCX_ERR_CUDA;
     attn_simt_kernel<T, Tout, 1><<<grid, kSimtBR * 1, smem, stream>>>(a);
   } else if (D == 64) {
-    cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (allow_smem(attn_simt_kernel<T, Tout, 2>, smem)) return RCX_ERR_CUDA;
     attn_simt_kernel<T, Tout, 2><<<grid, kSimtBR * 2, smem, stream>>>(a);
   } else {
-    cudaFuncSetAttribute(attn_simt_kernel<T, Tout, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (allow_smem(attn_simt_kernel<T, Tout, 4>, smem)) return RCX_ERR_CUDA;
     attn_simt_kernel<T, Tout, 4><<<grid, kSimtBR * 4, smem, stream>>>(a);
   }
   return launch_status();
