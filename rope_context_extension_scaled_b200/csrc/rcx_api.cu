@@ -504,11 +504,21 @@ int decode_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, c
   {
     dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
     LaunchScope scope(RCX_KERNEL_DECODE, stream);
-    switch (G) {
-      case 1: attn_decode_kernel<1><<<grid, kDecThreads, 0, stream>>>(a); break;
-      case 2: attn_decode_kernel<2><<<grid, kDecThreads, 0, stream>>>(a); break;
-      case 4: attn_decode_kernel<4><<<grid, kDecThreads, 0, stream>>>(a); break;
-      default: attn_decode_kernel<8><<<grid, kDecThreads, 0, stream>>>(a); break;
+    if (al(k, 16) && al(v, 16)) {
+      // tensor-core form: 16-byte rows of k and v for cp.async
+      auto kern = G == 1 ? attn_decode_mma_kernel<1>
+                : G == 2 ? attn_decode_mma_kernel<2>
+                : G == 4 ? attn_decode_mma_kernel<4>
+                         : attn_decode_mma_kernel<8>;
+      if (allow_smem(kern, kDmSmem)) return RCX_ERR_CUDA;
+      kern<<<grid, kDmWarps * 32, kDmSmem, stream>>>(a);
+    } else {
+      switch (G) {
+        case 1: attn_decode_kernel<1><<<grid, kDecThreads, 0, stream>>>(a); break;
+        case 2: attn_decode_kernel<2><<<grid, kDecThreads, 0, stream>>>(a); break;
+        case 4: attn_decode_kernel<4><<<grid, kDecThreads, 0, stream>>>(a); break;
+        default: attn_decode_kernel<8><<<grid, kDecThreads, 0, stream>>>(a); break;
+      }
     }
     if ((st = launch_status())) return st;
   }

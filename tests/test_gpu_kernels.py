@@ -323,6 +323,34 @@ def test_decode_split_kv_matches_oracle(B, Nk, Hq, Hkv, window, n_sink, qoff):
         assert err["inf_ok"] and err["o_max"] <= 2e-2 and err["lse_max"] <= 1e-3, err
 
 
+@pytest.mark.parametrize("Hq,Hkv,window,n_sink", [(8, 1, 0, 0), (16, 4, 300, 2)])
+def test_decode_8_byte_rows_matches_oracle(Hq, Hkv, window, n_sink):
+    """K and V rows 8- but not 16-byte aligned: the SIMT decode kernel."""
+    Nk = 2500
+    qf, _, _ = make_qkv(1, 1, Hq, Hkv, 128, torch.bfloat16, seed=25, device=DEV)
+    _, k, v = make_qkv(1, Nk, Hq, Hkv, 128, torch.bfloat16, seed=26, device=DEV)
+    inv, t = _lib.rope_freqs(_lib.YARN, 1e4, 128, 4096, 32768)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    kp = torch.zeros(1, Nk, Hkv, 132, dtype=torch.bfloat16, device=DEV)
+    vp = torch.zeros_like(kp)
+    kp[..., :128] = krot
+    vp[..., :128] = v
+    kv, vv = kp[..., :128], vp[..., :128]                       # row stride 264 bytes
+    o, lse = _lib.attn_decode_fwd(qf, kv, vv, window=window, n_sink=n_sink, temperature=t, q_index=Nk - 1,
+                                  inv_freq=inv, rope_flags=_lib.ROTATE_Q)
+    o2, lse2 = _lib.attn_decode_fwd(qf, krot, v, window=window, n_sink=n_sink, temperature=t, q_index=Nk - 1,
+                                    inv_freq=inv, rope_flags=_lib.ROTATE_Q)
+    torch.cuda.synchronize()
+    rows = {h: np.array([0]) for h in range(Hq)}
+    Or, Lr = oracle_rows(qf[0], k[0], v[0], inv, t, rows, window, n_sink, q_start=Nk - 1, k_start=0)
+    for oo, ll in ((o, lse), (o2, lse2)):
+        Og = {h: np64(oo[0, 0, h, :])[None] for h in range(Hq)}
+        Lg = {h: np.array([float(ll[0, h, 0])]) for h in range(Hq)}
+        err = errors(Og, Lg, Or, Lr)
+        assert err["inf_ok"] and err["o_max"] <= 2e-2 and err["lse_max"] <= 1e-3, err
+
+
 def test_decode_rejects_rotate_k_and_bad_group():
     q, k, v = make_qkv(1, 1, 6, 2, 128, torch.bfloat16, seed=22, device=DEV)   # G = 3
     _, kc, vc = make_qkv(1, 64, 6, 2, 128, torch.bfloat16, seed=23, device=DEV)
