@@ -141,25 +141,34 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, shapes from the instruction descriptor.
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
+// D[tmem] (+)= A[smem] * B[smem]^T (SS) and D[tmem] (+)= A[tmem] * B[smem]
+// (TS), shapes from the instruction descriptor, with each shared-memory
+// descriptor passed as its two 32-bit words.  The low word holds start
+// address >> 4 in bits 0-13 and LBO >> 4 in bits 16-29; shared memory is
+// below 256 KB, so adding (byte offset >> 4) to the low word steps the start
+// address without carrying into LBO.  The issuing thread then spends a few
+// instructions per MMA: it shares its SM sub-partition with two softmax warps,
+// and MMA issue is on the kernel's critical path.
+__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem].
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -450,21 +459,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t id_qk = idesc_bf16(false);
       constexpr uint32_t id_pv = idesc_bf16(true);
       ok = ok && mbar_wait(BAR(B_QREADY + 0), 0, abort_flag) && mbar_wait(BAR(B_QREADY + 1), 0, abort_flag);
+      // descriptor words, built once: Q (K-major, per slot), K and V (per stage)
+      const uint32_t d_hi = (uint32_t)(sw128_desc(sbase, 16, 1024) >> 32);
+      const uint32_t q_lo[2] = {(uint32_t)sw128_desc(sbase + kSmQ, 16, 1024),
+                                (uint32_t)sw128_desc(sbase + kSmQ + kTileBytes, 16, 1024)};
+      const uint32_t k_lo = (uint32_t)sw128_desc(sbase + kSmK, 16, 1024);
+      const uint32_t v_lo = (uint32_t)sw128_desc(sbase + kSmV, kHalfTileBytes, 1024);
       auto issue_s = [&](int s, int st) {
-        const uint32_t qa = sbase + kSmQ + s * kTileBytes;
-        const uint32_t ka = sbase + kSmK + st * kTileBytes;
+        const uint32_t a0 = q_lo[s], b0 = k_lo + st * (kTileBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcD / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kHalfTileBytes + (kk % 4) * 32;
-          umma_ss(tS[s], sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_qk, kk > 0);
+          const uint32_t off = ((kk / 4) * kHalfTileBytes + (kk % 4) * 32) >> 4;
+          umma_ss_w(tS[s], a0 + off, b0 + off, d_hi, id_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int s, int st, bool first_tile) {
-        const uint32_t va = sbase + kSmV + st * kTileBytes;
+        const uint32_t b0 = v_lo + st * (kTileBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcBN / 16; ++kk)
-          umma_ts(tO[s], tS[s] + kk * 8, sw128_desc(va + kk * 2048, kHalfTileBytes, 1024), id_pv,
-                  (!first_tile || kk > 0) ? 1u : 0u);
+          umma_ts_w(tO[s], tS[s] + kk * 8, b0 + kk * (2048 >> 4), d_hi, id_pv, (!first_tile || kk > 0) ? 1u : 0u);
       };
       if (ok && n > 0) {
         ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag);
