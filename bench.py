@@ -40,7 +40,7 @@ METRIC = "causal attention fwd TFLOP/s and % of B200 BF16 tensor peak at 128K an
 # every attention launch of one step of the same command (summary and command in
 # profiles/attn_tc_traffic_llama3_70b_1m_ring.md).  Valid for the attention
 # kernel as captured; re-take it when the kernel changes.
-ATTN_TRAFFIC_PER_LAUNCH = {"llama3_70b_1m_ring": 3.743e9}
+ATTN_TRAFFIC_PER_LAUNCH = {"llama3_70b_1m_ring": 3.729e9}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
