@@ -342,6 +342,41 @@ def merge(o_a, lse_a, o_b, lse_b):
 
 
 # --------------------------------------------------------------------------
+# Int8 KV cache
+# --------------------------------------------------------------------------
+
+def quantize_kv_int8(x):
+    """Symmetric int8 codes and one fp32 scale per (..., row) of a KV cache.
+
+    "Context window extension: 4K to 1M" section 6.1 stores the KV cache in
+    INT8 instead of 16-bit floats to halve its memory (the "Context Extension"
+    concept page lists the same compression in its KV-cache table).  The pages
+    fix no format; the reading taken is the plainest symmetric one, per row of
+    d values (one token of one KV head):
+        amax = max |x|,  scale = amax / 127,  code = rint(x * (127 / amax)),
+    clamped to [-127, 127] (all zero when amax = 0).  The codes are integers
+    decided by floating point, so they are computed in IEEE fp32 (division,
+    product, round-half-to-even), the precision the device uses too.
+    x: [..., d] (the values the device sees); returns (codes int8 [..., d],
+    scale float32 [...]).
+    """
+    xf = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(xf), axis=-1).astype(np.float32)
+    live = amax > 0
+    safe = np.where(live, amax, np.float32(1)).astype(np.float32)
+    scale = np.where(live, safe / np.float32(127), np.float32(0)).astype(np.float32)
+    inv = np.where(live, np.float32(127) / safe, np.float32(0)).astype(np.float32)
+    prod = (xf * inv[..., None]).astype(np.float32)
+    codes = np.clip(np.rint(prod), -127, 127).astype(np.int8)
+    return codes, scale
+
+
+def dequantize_kv_int8(codes, scale):
+    """The cache values an int8 KV cache stands for: code * scale (float64)."""
+    return np.asarray(codes, dtype=np.float64) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+# --------------------------------------------------------------------------
 # Ring order
 # --------------------------------------------------------------------------
 

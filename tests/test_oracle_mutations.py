@@ -34,6 +34,10 @@ MUTATIONS = [
     ("s = seq_len / L_train", "s = L_train / seq_len"),
     ("total += min(n_sink, lo)", "total += n_sink"),
     ("return rope_theta(base, d) / lam", "return rope_theta(base, d) * lam"),
+    ("scale = np.where(live, safe / np.float32(127), np.float32(0))", "scale = np.where(live, safe / np.float32(128), np.float32(0))"),
+    ("codes = np.clip(np.rint(prod), -127, 127)", "codes = np.clip(np.floor(prod + 0.5), -127, 127)"),
+    ("codes = np.clip(np.rint(prod), -127, 127)", "codes = np.clip(np.trunc(prod), -127, 127)"),
+    ("inv = np.where(live, np.float32(127) / safe, np.float32(0))", "inv = np.where(live, np.float32(127.5) / safe, np.float32(0))"),
 ]
 
 

@@ -470,3 +470,47 @@ def test_ring_ordered_blocks_then_merge_equal_full():
         O[rows], L[:, rows] = acc_o, acc_l.T
     np.testing.assert_allclose(O, full[0], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(L, full[1], rtol=1e-13)
+
+
+# --------------------------------------------------------------- int8 KV cache
+
+def test_int8_codes_exact_for_representable_rows():
+    """Rows k * 2^-e with integer k in [-127, 127] and |k|max = 127: the scale
+    is 2^-e exactly, the codes are k and dequantisation gives the row back."""
+    rng = np.random.default_rng(40)
+    for e in (0, 3, 9):
+        k = rng.integers(-127, 128, size=(5, 128))
+        k[:, 7] = 127
+        k[2, 7] = -127
+        x = k.astype(np.float64) * 2.0 ** -e
+        codes, scale = orc.quantize_kv_int8(x)
+        assert np.array_equal(codes.astype(np.int64), k)
+        assert np.all(scale == np.float32(2.0 ** -e))
+        assert np.array_equal(orc.dequantize_kv_int8(codes, scale), x)
+
+
+def test_int8_ties_round_to_even_and_sign_symmetry():
+    # amax = 127 -> 127/amax = 1, so code = rint(x): x.5 ties go to the even code
+    x = np.array([[127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, 126.5] + [0.0] * 120])
+    codes, scale = orc.quantize_kv_int8(x)
+    assert scale[0] == np.float32(1.0)
+    assert codes[0, :8].tolist() == [127, 2, 4, -2, -4, 0, 2, 126]
+    c2, s2 = orc.quantize_kv_int8(-x)
+    assert np.array_equal(c2, -codes) and np.array_equal(s2, scale)
+
+
+def test_int8_zero_row_and_error_bound():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((64, 4, 128)).astype(np.float32) * rng.uniform(1e-3, 50.0, (64, 4, 1)).astype(np.float32)
+    x[3, 1] = 0.0
+    codes, scale = orc.quantize_kv_int8(x)
+    assert scale[3, 1] == 0.0 and not codes[3, 1].any()
+    live = scale > 0
+    # the largest magnitude of every non-zero row maps to +-127
+    assert np.all(np.abs(codes.astype(np.int64)).max(axis=-1)[live] == 127)
+    # round-to-nearest: |x - code * scale| <= scale / 2 (plus fp32 rounding of 127/amax)
+    err = np.abs(x.astype(np.float64) - orc.dequantize_kv_int8(codes, scale))
+    bound = scale.astype(np.float64)[..., None] * (0.5 + 1e-5) + 1e-6 * np.abs(x)
+    assert np.all(err <= bound)
+    # and the scale is amax / 127
+    np.testing.assert_allclose(scale, np.abs(x).max(axis=-1) / 127.0, rtol=1e-7)
