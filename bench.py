@@ -384,7 +384,23 @@ def run_ours(args, w):
                   "ms": d_ms, "gbs": kv_bytes / (d_ms * 1e-3) / 1e9,
                   "pct_hbm": 100.0 * kv_bytes / (d_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                   "tokens_per_s": world * w.B / (d_ms * 1e-3)}
-        del qd, od, ld, wsd
+        # the same decode over the int8 copy of the cache (codes made outside the timed region)
+        kc, ks = _lib.kv_quantize_int8(k)
+        vc, vs = _lib.kv_quantize_int8(v)
+        ws8 = torch.empty(max(_lib.load().rcx_attn_decode_int8_workspace_size(_lib.view(qd), _lib.view(kc)), 256),
+                          dtype=torch.uint8, device="cuda")
+
+        def dstep8():
+            _lib.attn_decode_int8_fwd(qd, kc, ks, vc, vs, od, ld, window=w.window, n_sink=w.n_sink,
+                                      temperature=t_d, q_index=w.N - 1, inv_freq=inv_d, rope_flags=_lib.ROTATE_Q,
+                                      workspace=ws8)
+        d8_ms = time_steps(dstep8, 20, 5, stream, dist, world)
+        kv8_bytes = 2.0 * (kc.numel() + 4 * ks.numel())
+        decode["int8_cache"] = {"ms": d8_ms, "gbs": kv8_bytes / (d8_ms * 1e-3) / 1e9,
+                                "pct_hbm": 100.0 * kv8_bytes / (d8_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "tokens_per_s": world * w.B / (d8_ms * 1e-3),
+                                "bytes_per_step": kv8_bytes}
+        del qd, od, ld, wsd, kc, ks, vc, vs, ws8
     peak_key = "bf16_tflops_sustained" if ms > 1000 else "bf16_tflops"
     peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
     achieved = flops / (attn_ms * 1e-3) / 1e12

@@ -39,7 +39,7 @@ typedef enum {
     RCX_ERR_DEVICE_TIMEOUT = -5  /* a device-side bounded wait gave up         */
 } rcx_status;
 
-typedef enum { RCX_F32 = 0, RCX_BF16 = 1 } rcx_dtype;
+typedef enum { RCX_F32 = 0, RCX_BF16 = 1, RCX_I8 = 2 /* int8 KV-cache codes only */ } rcx_dtype;
 
 /* RoPE frequency schedules (see rcx_rope_freqs). */
 typedef enum {
@@ -187,6 +187,49 @@ int rcx_attn_decode_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, 
                         int64_t window, int64_t n_sink, double temperature, int64_t q_index,
                         const int64_t* positions, int64_t n_positions, const double* inv_freq,
                         int rope_flags, void* workspace, int64_t workspace_bytes, void* stream);
+
+/*
+ * rcx_kv_quantize_int8 -- int8 KV-cache codes of a bf16 cache
+ * ("Context window extension: 4K to 1M" 6.1: the KV cache held in INT8
+ * instead of 16-bit floats, half the memory; the "Context Extension" concept
+ * page lists the same compression).  Per row of d = 128 values (one token of
+ * one head): amax = max |x|, scale = amax / 127, code = rint(x * (127 / amax))
+ * clamped to [-127, 127]; a zero row gets scale 0 and zero codes.  The codes
+ * are decided in IEEE fp32 (correctly rounded division and product,
+ * round-half-to-even), so any fp32 implementation of the same rule gives the
+ * same bytes.
+ *
+ * x: [B, N, H, 128] bf16, 8-byte aligned rows.  codes: [B, N, H, 128]
+ * RCX_I8, same shape, 4-byte aligned rows.  scale: device fp32 [B, N, H],
+ * contiguous (row (b, n, h) at (b * N + n) * H + h), caller-owned.  Memory
+ * bound: reads x once, writes codes and scales once.  Launches are timed
+ * under RCX_KERNEL_DECODE.
+ */
+int rcx_kv_quantize_int8(rcx_tensor x, rcx_tensor codes, float* scale, void* stream);
+
+/*
+ * rcx_attn_decode_int8_fwd -- rcx_attn_decode_fwd over an int8 KV cache made
+ * by rcx_kv_quantize_int8: key j of KV head h stands for k_codes[j] *
+ * k_scale[j, h] (and likewise V).  Same query, mask, GQA, temperature, LSE,
+ * rope_flags and split-KV merge as rcx_attn_decode_fwd; the codes are
+ * dequantised in the tile load and the contractions run in fp16 with fp32
+ * accumulation, so |rotated q| and the dequantised V must stay below the fp16
+ * range (65504).
+ *
+ * q, o: [B, 1, Hq, 128] (q bf16; o bf16 or f32); k, v: [B, Nk, Hkv, 128]
+ * RCX_I8, 16-byte aligned rows (base and strides multiples of 16 bytes);
+ * k_scale, v_scale: device fp32 [B, Nk, Hkv] contiguous; Hq / Hkv in
+ * {1, 2, 4, 8}; lse: [B, Hq, 1, 1] fp32 or ptr NULL.  workspace: device
+ * buffer of rcx_attn_decode_int8_workspace_size(q, k) bytes, 256-byte
+ * aligned, caller-owned.  Memory-bound: reads each code and scale once (half
+ * the bytes of the bf16 cache).
+ */
+int64_t rcx_attn_decode_int8_workspace_size(rcx_tensor q, rcx_tensor k);
+int rcx_attn_decode_int8_fwd(rcx_tensor q, rcx_tensor k, const float* k_scale, rcx_tensor v,
+                             const float* v_scale, rcx_tensor o, rcx_tensor lse, int64_t window,
+                             int64_t n_sink, double temperature, int64_t q_index,
+                             const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                             int rope_flags, void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
  * rcx_merge_partials -- LSE-weighted merge of two partial results over

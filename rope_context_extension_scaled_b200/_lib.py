@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "librcx.so")
 
 RCX_OK, RCX_ERR_INVALID_ARG, RCX_ERR_UNSUPPORTED, RCX_ERR_ALIGNMENT, RCX_ERR_CUDA, RCX_ERR_DEVICE_TIMEOUT = \
     0, -1, -2, -3, -4, -5
-RCX_F32, RCX_BF16 = 0, 1
+RCX_F32, RCX_BF16, RCX_I8 = 0, 1, 2
 PLAIN, PI, NTK, DYN_NTK, NTK_PARTS, YARN = range(6)
 ROTATE_Q, ROTATE_K = 1, 2
 
@@ -31,7 +31,8 @@ EXPORTS = (
     "rcx_ring_attn_fwd", "rcx_ring_attn_fwd_host", "rcx_device_status",
     "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
     "rcx_ring_attn_fwd_noalloc", "rcx_rope_freqs_per_pair", "rcx_attn_decode_workspace_size",
-    "rcx_attn_decode_fwd",
+    "rcx_attn_decode_fwd", "rcx_kv_quantize_int8", "rcx_attn_decode_int8_workspace_size",
+    "rcx_attn_decode_int8_fwd",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20   # RCX_NOALLOC_SCRATCH_BYTES in include/rcx.h
 KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3, "decode": 4}
@@ -73,6 +74,12 @@ def load():
     lib.rcx_attn_decode_workspace_size.restype = i64
     lib.rcx_attn_decode_fwd.argtypes = [T, T, T, T, T, i64, i64, f64, i64, vp, i64, pd, ctypes.c_int, vp, i64, vp]
     lib.rcx_attn_decode_fwd.restype = ctypes.c_int
+    lib.rcx_kv_quantize_int8.argtypes = [T, T, vp, vp]
+    lib.rcx_attn_decode_int8_workspace_size.argtypes = [T, T]
+    lib.rcx_attn_decode_int8_workspace_size.restype = i64
+    lib.rcx_attn_decode_int8_fwd.argtypes = [T, T, vp, T, vp, T, T, i64, i64, f64, i64, vp, i64, pd, ctypes.c_int,
+                                             vp, i64, vp]
+    lib.rcx_attn_decode_int8_fwd.restype = ctypes.c_int
     lib.rcx_attn_blockwise_fwd.argtypes = [T, T, T, T, T, i64, i64, i64, f64, i64, i64, vp, i64, pd,
                                            ctypes.c_int, vp]
     lib.rcx_merge_partials.argtypes = [T, T, T, T, T, T, vp]
@@ -109,6 +116,8 @@ def _dtype_code(t: torch.Tensor):
         return RCX_F32
     if t.dtype == torch.bfloat16:
         return RCX_BF16
+    if t.dtype == torch.int8:
+        return RCX_I8
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -301,6 +310,49 @@ def ring_attn_fwd_noalloc(q, k, v, o, lse=None, kv_block=0, window=0, n_sink=0, 
                                           int(window), int(n_sink), float(temperature), pp, npos, fp,
                                           int(rope_flags), _stream(q.device))
     _check(st, "rcx_ring_attn_fwd_noalloc")
+    return o, lse
+
+
+def kv_quantize_int8(x, codes=None, scale=None):
+    """Int8 codes [B, N, H, 128] and fp32 scales [B, N, H] of a bf16 cache x."""
+    B, N, H, _ = x.shape
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scale is None:
+        scale = torch.empty(B, N, H, dtype=torch.float32, device=x.device)
+    if not scale.is_contiguous() or scale.dtype != torch.float32 or tuple(scale.shape) != (B, N, H):
+        raise ValueError("scale must be a contiguous float32 [B, N, H] tensor")
+    st = load().rcx_kv_quantize_int8(view(x), view(codes), ctypes.c_void_p(scale.data_ptr()), _stream(x.device))
+    _check(st, "rcx_kv_quantize_int8")
+    return codes, scale
+
+
+def attn_decode_int8_fwd(q, k, k_scale, v, v_scale, o=None, lse=None, window=0, n_sink=0, temperature=1.0,
+                         q_index=None, positions=None, inv_freq=None, rope_flags=0, workspace=None, want_lse=True):
+    """attn_decode_fwd over an int8 cache (codes k, v [B, Nk, Hkv, 128], scales [B, Nk, Hkv])."""
+    B, _, H, D = q.shape
+    if q_index is None:
+        q_index = k.shape[1] - 1
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, 1, dtype=torch.float32, device=q.device)
+    for sc in (k_scale, v_scale):
+        if not sc.is_contiguous() or sc.dtype != torch.float32 or tuple(sc.shape) != tuple(k.shape[:3]):
+            raise ValueError("scales must be contiguous float32 [B, Nk, Hkv] tensors")
+    need = load().rcx_attn_decode_int8_workspace_size(view(q), view(k))
+    if need < 0:
+        raise RcxError(RCX_ERR_INVALID_ARG, "rcx_attn_decode_int8_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    arr, fp = _freq_ptr(inv_freq)
+    pp, npos = _pos(positions)
+    st = load().rcx_attn_decode_int8_fwd(view(q), view(k), ctypes.c_void_p(k_scale.data_ptr()), view(v),
+                                         ctypes.c_void_p(v_scale.data_ptr()), view(o), lse_view(lse), int(window),
+                                         int(n_sink), float(temperature), int(q_index), pp, npos, fp,
+                                         int(rope_flags), ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                         _stream(q.device))
+    _check(st, "rcx_attn_decode_int8_fwd")
     return o, lse
 
 

@@ -1,0 +1,364 @@
+// Int8 KV cache: per-row quantisation and decode attention over the codes.
+//
+// "Context window extension: 4K to 1M" section 6.1 keeps the KV cache in INT8
+// instead of 16-bit floats, halving its memory; the "Context Extension"
+// concept page lists the same compression in its KV-cache table.  Format
+// (the plainest symmetric reading; the pages fix none): one fp32 scale per
+// row of d = 128 values (one token of one KV head), scale = amax / 127 and
+// code = rint(x * (127 / amax)) in [-127, 127], all decided in IEEE fp32.
+//
+// Decode over the codes follows attn_decode_mma_kernel (16-key tiles per
+// warp, three cp.async stages, transposed mma.sync with the G <= 8 query heads
+// as the MMA columns) with the dequantisation in the tile load:
+//  * the MMAs run in fp16 (m16n8k16, fp32 accumulate), because an int8 code
+//    becomes an exact fp16 in three integer/half instructions: the byte with
+//    its sign bit flipped (u = code + 128) is placed under the exponent
+//    pattern of 1024, which reads as 1024 + u, and 1152 is subtracted;
+//  * K codes go into S^T = Kq Q^T unscaled; each key's scale then multiplies
+//    its row of S^T in fp32;
+//  * V codes go into O^T += Vq^T P'^T unscaled, with each key's V scale folded
+//    into P: P' = p * s_v / s_max, where s_max is the largest V scale the warp
+//    has met so far (so P' stays in [0, 1], clear of fp16 subnormals).  When
+//    s_max grows, O is rescaled together with the online-softmax correction,
+//    and O * s_max is the warp's result.
+// K row reads use the same d permutation trick as the bf16 kernel's first
+// form: lane c of a row group takes dims [32c, 32c + 32) of the key in order,
+// and Q is laid out with the same permutation, so every dot product is
+// unchanged.  The V^T operand rows (d) are permuted too: lane g's rows are
+// dims [16g, 16g + 16), and the merge writes them back in natural order.
+#pragma once
+#include <cuda_fp16.h>
+#include "attn_decode.cuh"
+
+namespace rcx {
+
+// ---------------------------------------------------------------- quantise
+
+struct QuantArgs {
+  View4 x;          // bf16 [B, N, H, 128]
+  View4 c;          // int8 [B, N, H, 128]
+  float* scale;     // [B, N, H] contiguous
+  int64_t rows;     // B * N * H
+};
+
+// One warp per row; lane l holds dims 4l .. 4l + 3.  A warp takes kQRows rows
+// per pass (grid-strided) and issues all their loads before any arithmetic.
+constexpr int kQRows = 4;
+
+__global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const QuantArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
+  const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  for (int64_t r0 = w0; r0 < a.rows; r0 += kQRows * nwarps) {
+    uint2 u[kQRows];
+    int64_t off_c[kQRows];
+#pragma unroll
+    for (int i = 0; i < kQRows; ++i) {
+      const int64_t r = r0 + i * nwarps;
+      const int64_t rr = r < a.rows ? r : r0;
+      const int64_t h = rr % a.x.H;
+      const int64_t n = (rr / a.x.H) % a.x.N;
+      const int64_t b = rr / (a.x.H * a.x.N);
+      const __nv_bfloat16* xp = reinterpret_cast<const __nv_bfloat16*>(a.x.ptr) + b * a.x.sb + n * a.x.sn +
+                                h * a.x.sh + 4 * lane;
+      u[i] = *reinterpret_cast<const uint2*>(xp);
+      off_c[i] = b * a.c.sb + n * a.c.sn + h * a.c.sh + 4 * lane;
+    }
+#pragma unroll
+    for (int i = 0; i < kQRows; ++i) {
+      const int64_t r = r0 + i * nwarps;
+      if (r >= a.rows) break;                      // warp-uniform
+      const float2 x01 = bf2_to_f2(u[i].x), x23 = bf2_to_f2(u[i].y);
+      const float v[4] = {x01.x, x01.y, x23.x, x23.y};
+      float am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+      const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int q = __float2int_rn(__fmul_rn(v[e], inv));
+        q = q > 127 ? 127 : (q < -127 ? -127 : q);
+        packed |= (uint32_t)(q & 0xff) << (8 * e);
+      }
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(a.c.ptr) + off_c[i]) = packed;
+      if (lane == 0) a.scale[r] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- decode
+
+constexpr int kDqWarps = 4;
+constexpr int kDqStages = 3;
+constexpr int kDqRow = 144;                                  // 128-byte code row + 16 pad (banks)
+constexpr int kDqTile = 16 * kDqRow;                         // one 16-key K or V tile
+constexpr int kDqStage = 2 * kDqTile + 2 * 64;               // K, V, 16 K scales, 16 V scales
+constexpr int kDqSmem = kDqWarps * kDqStages * kDqStage;     // 56,832 B: three CTAs per SM
+static_assert(kDqSmem >= kDqWarps * kDecMaxG * 128 * 4, "merge area aliases the stage buffers");
+
+__device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Two int8 codes (bytes 0 and 2 of u ^ 0x80808080 selected by sel) -> exact fp16 pair.
+__device__ __forceinline__ uint32_t codes_to_h2(uint32_t u_flipped, uint32_t sel) {
+  const uint32_t h = __byte_perm(u_flipped, 0x64646464u, sel);      // halves 0x64uu = 1024 + u
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h), __half2half2(__ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&r);                    // 0x6480 = 1152
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const DecodeArgs a,
+                                                                        const float* __restrict__ k_scale,
+                                                                        const float* __restrict__ v_scale) {
+  extern __shared__ __align__(128) uint8_t dq_smem[];
+  __shared__ float sm_m[kDqWarps][kDecMaxG], sm_l[kDqWarps][kDecMaxG];
+  const int split = blockIdx.x;
+  const int hk = blockIdx.y;
+  const int64_t b = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = lane >> 2, c = lane & 3;
+
+  // ---- Q^T operand (fp16): head g, dims 32c + 4kc + {0, 1} (b0) and {2, 3} (b1)
+  uint32_t qb[8][2];
+  if (g < G) {
+    const __nv_bfloat16* qp =
+        reinterpret_cast<const __nv_bfloat16*>(a.q.ptr) + b * a.q.sb + (int64_t)(hk * G + g) * a.q.sh + 32 * c;
+    const int64_t qpos = a.positions ? a.positions[a.q_index] : a.q_index;
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int d0 = 4 * kc + 2 * hf;
+        float2 x = bf2_to_f2(*reinterpret_cast<const uint32_t*>(qp + d0));
+        if (a.rope_q) {
+          float cs, sn;
+          rope_cos_sin(qpos, a.f.theta[16 * c + (d0 >> 1)], cs, sn);
+          x = make_float2(x.x * cs - x.y * sn, x.x * sn + x.y * cs);
+        }
+        qb[kc][hf] = f2_to_h2(x.x, x.y);
+      }
+  } else {
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) qb[kc][0] = qb[kc][1] = 0u;
+  }
+
+  // ---- this warp's key range, in 16-key tiles from k_lo
+  const int64_t Nk = a.k.N, Hkv = a.k.H;
+  const int64_t s_lo = (int64_t)split * a.keys_per_split;
+  const int64_t s_hi = min(Nk, s_lo + a.keys_per_split);
+  const int64_t per_warp = ((s_hi - s_lo + kDqWarps - 1) / kDqWarps + 15) / 16 * 16;
+  const int64_t k_lo = s_lo + warp * per_warp;
+  const int64_t k_hi = min(s_hi, k_lo + per_warp);
+  const int64_t qi = a.q_index;
+  auto next_visible = [&](int64_t t) {
+    while (t < k_hi && !tile_any_visible(qi, qi, t, min(t + 15, k_hi - 1), a.window, a.n_sink)) {
+      if (t > qi) return k_hi;
+      t += 16;
+    }
+    return t < k_hi ? t : k_hi;
+  };
+
+  const int8_t* kbase = reinterpret_cast<const int8_t*>(a.k.ptr) + b * a.k.sb + hk * a.k.sh;
+  const int8_t* vbase = reinterpret_cast<const int8_t*>(a.v.ptr) + b * a.v.sb + hk * a.v.sh;
+  const float* ksc = k_scale + b * Nk * Hkv + hk;            // key j: ksc[j * Hkv]
+  const float* vsc = v_scale + b * Nk * Hkv + hk;
+  uint8_t* wptr = dq_smem + warp * kDqStages * kDqStage;
+  const uint32_t wbuf = static_cast<uint32_t>(__cvta_generic_to_shared(wptr));
+  // codes and scales of keys t .. t + 15 -> stage st (keys past the range are zero-filled)
+  auto issue = [&](int64_t t, int st) {
+    if (t < k_hi) {
+      const uint32_t ks = wbuf + st * kDqStage;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = lane + 32 * i;
+        const int key = e >> 3, col = e & 7;
+        const int64_t j = t + key;
+        const bool ok = j < k_hi;
+        const int64_t jj = ok ? j : t;
+        const int bytes = ok ? 16 : 0;
+        const uint32_t off = key * kDqRow + col * 16;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ks + off),
+                     "l"(kbase + jj * a.k.sn + col * 16), "r"(bytes)
+                     : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ks + kDqTile + off),
+                     "l"(vbase + jj * a.v.sn + col * 16), "r"(bytes)
+                     : "memory");
+      }
+      {
+        const int key = lane & 15;
+        const int64_t j = t + key;
+        const bool ok = j < k_hi;
+        const float* src = (lane < 16 ? ksc : vsc) + (ok ? j : t) * Hkv;
+        const uint32_t dst = ks + 2 * kDqTile + (lane < 16 ? 0 : 64) + key * 4;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(ok ? 4 : 0)
+                     : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // heads 2c, 2c + 1 (l: this lane's share)
+  float smax = 0.f;                                         // largest V scale met so far
+  float o[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+
+  int64_t t0 = next_visible(k_lo);
+  int64_t t1 = t0 < k_hi ? next_visible(t0 + 16) : k_hi;
+  issue(t0, 0);
+  issue(t1, 1);
+  int st = 0;
+  while (t0 < k_hi) {
+    const int64_t t2 = t1 < k_hi ? next_visible(t1 + 16) : k_hi;
+    issue(t2, st == 0 ? 2 : st - 1);
+    asm volatile("cp.async.wait_group 2;" ::: "memory");
+    __syncwarp();
+    const uint8_t* ks = wptr + st * kDqStage;
+    const uint8_t* vs = ks + kDqTile;
+    const float* sk = reinterpret_cast<const float*>(ks + 2 * kDqTile);
+    const float* sv_ = sk + 16;
+    // S^T = Kq Q^T: K rows g and g + 8, dims [32c, 32c + 32)
+    uint32_t kw[2][8];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const uint4 u0 = *reinterpret_cast<const uint4*>(ks + (g + 8 * r) * kDqRow + 32 * c);
+      const uint4 u1 = *reinterpret_cast<const uint4*>(ks + (g + 8 * r) * kDqRow + 32 * c + 16);
+      kw[r][0] = u0.x; kw[r][1] = u0.y; kw[r][2] = u0.z; kw[r][3] = u0.w;
+      kw[r][4] = u1.x; kw[r][5] = u1.y; kw[r][6] = u1.z; kw[r][7] = u1.w;
+    }
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) {
+      const uint32_t fa = kw[0][kc] ^ 0x80808080u, fb = kw[1][kc] ^ 0x80808080u;
+      const uint32_t af[4] = {codes_to_h2(fa, 0x4140), codes_to_h2(fb, 0x4140), codes_to_h2(fa, 0x4342),
+                              codes_to_h2(fb, 0x4342)};
+      mma_f16_16816(sacc, af, qb[kc][0], qb[kc][1]);
+    }
+    // key scales, online softmax per head over keys t0 + g, t0 + g + 8
+    const float ska = sk[g], skb = sk[g + 8];
+    const float sva = sv_[g], svb = sv_[g + 8];
+    float tmax = fmaxf(sva, svb);
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+    const float smax_new = fmaxf(smax, tmax);
+    const float ratio = smax_new > 0.f ? smax / smax_new : 1.f;
+    const float inv_smax = smax_new > 0.f ? 1.f / smax_new : 0.f;
+    smax = smax_new;
+    const int64_t ja = t0 + g, jb = t0 + g + 8;
+    const bool va = ja < k_hi && mask_visible(qi, ja, a.window, a.n_sink);
+    const bool vb = jb < k_hi && mask_visible(qi, jb, a.window, a.n_sink);
+    float sv[4];
+    sv[0] = va ? sacc[0] * ska * a.scale_log2 : -INFINITY;
+    sv[1] = va ? sacc[1] * ska * a.scale_log2 : -INFINITY;
+    sv[2] = vb ? sacc[2] * skb * a.scale_log2 : -INFINITY;
+    sv[3] = vb ? sacc[3] * skb * a.scale_log2 : -INFINITY;
+    float p[4], beta[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float mx = fmaxf(sv[h], sv[h + 2]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m[h], mx);
+      const float mref = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = dec_exp2(m[h] - mref);
+      p[h] = dec_exp2(sv[h] - mref);
+      p[h + 2] = dec_exp2(sv[h + 2] - mref);
+      l[h] = l[h] * alpha + (p[h] + p[h + 2]);
+      m[h] = m_new;
+      beta[h] = alpha * ratio;
+    }
+    // P' = p * s_v / s_max, transposed into the B operand of the P V product
+    const float wa = sva * inv_smax, wb = svb * inv_smax;
+    const uint32_t pb0 = movmatrix_t(f2_to_h2(p[0] * wa, p[1] * wa));   // keys 2c, 2c + 1 of head g
+    const uint32_t pb1 = movmatrix_t(f2_to_h2(p[2] * wb, p[3] * wb));   // keys 2c + 8, 2c + 9
+    // O^T = beta O^T + Vq^T P'^T: V rows 2c, 2c + 1, 2c + 8, 2c + 9, dims [16g, 16g + 16)
+    uint4 vr[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int key = 2 * c + (i & 1) + 8 * (i >> 1);
+      vr[i] = *reinterpret_cast<const uint4*>(vs + key * kDqRow + 16 * g);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      o[mt][0] *= beta[0];
+      o[mt][1] *= beta[1];
+      o[mt][2] *= beta[0];
+      o[mt][3] *= beta[1];
+      // operand rows: dim 16g + 2mt (row g) and 16g + 2mt + 1 (row g + 8)
+      const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;   // bytes j, j + 1 of two keys, interleaved
+      const int wi = mt >> 1;
+      auto word = [](const uint4& u, int i) { return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w; };
+      const uint32_t lo = __byte_perm(word(vr[0], wi), word(vr[1], wi), sel) ^ 0x80808080u;   // keys 2c, 2c+1
+      const uint32_t hi = __byte_perm(word(vr[2], wi), word(vr[3], wi), sel) ^ 0x80808080u;   // keys 2c+8, 2c+9
+      const uint32_t af[4] = {codes_to_h2(lo, 0x4140), codes_to_h2(lo, 0x4342), codes_to_h2(hi, 0x4140),
+                              codes_to_h2(hi, 0x4342)};
+      mma_f16_16816(o[mt], af, pb0, pb1);
+    }
+    __syncwarp();   // stage st is refilled two iterations on
+    st = st == kDqStages - 1 ? 0 : st + 1;
+    t0 = t1;
+    t1 = t2;
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+  // ---- merge the warps' states in shared memory (aliases the stage buffers)
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 4);
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 8);
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 16);
+  }
+  __syncthreads();
+  float* sm_o = reinterpret_cast<float*>(dq_smem);   // [warps][kDecMaxG][128]
+  if (g == 0) {
+    sm_m[warp][2 * c] = m[0];
+    sm_m[warp][2 * c + 1] = m[1];
+    sm_l[warp][2 * c] = l[0];
+    sm_l[warp][2 * c + 1] = l[1];
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    // C rows: g -> dim 16g + 2mt, g + 8 -> dim 16g + 2mt + 1; columns: heads 2c, 2c + 1
+    float* w0 = sm_o + (warp * kDecMaxG + 2 * c) * 128 + 16 * g + 2 * mt;
+    w0[0] = o[mt][0] * smax;
+    w0[128] = o[mt][1] * smax;
+    w0[1] = o[mt][2] * smax;
+    w0[128 + 1] = o[mt][3] * smax;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * 128; e += blockDim.x) {
+    const int hh = e / 128, dd = e % 128;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDqWarps; ++w) mm = fmaxf(mm, sm_m[w][hh]);
+    const float mr = mm == -INFINITY ? 0.f : mm;
+    float lt = 0.f, ot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDqWarps; ++w) {
+      const float wgt = dec_exp2(sm_m[w][hh] - mr);
+      lt += wgt * sm_l[w][hh];
+      ot += wgt * sm_o[(w * kDecMaxG + hh) * 128 + dd];
+    }
+    const int64_t hq = (int64_t)hk * G + hh;
+    const int64_t pidx = ((int64_t)split * a.q.B + b) * a.q.H + hq;
+    a.part_o[pidx * 128 + dd] = lt > 0.f ? ot / lt : 0.f;
+    if (dd == 0) a.part_lse[pidx] = lt > 0.f ? (mr + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+  }
+}
+
+}  // namespace rcx

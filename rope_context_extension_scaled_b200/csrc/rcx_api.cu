@@ -18,6 +18,7 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "attn_decode.cuh"
+#include "kv_int8.cuh"
 #include "rope_freqs.inc"
 
 using namespace rcx;
@@ -81,7 +82,7 @@ constexpr int kAbiVersion = 100;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-inline int elem_size(int dtype) { return dtype == RCX_BF16 ? 2 : 4; }
+inline int elem_size(int dtype) { return dtype == RCX_BF16 ? 2 : dtype == RCX_I8 ? 1 : 4; }
 
 int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
@@ -437,10 +438,11 @@ struct DecodePlan {
   int64_t keys_per_split, off_lse, total;
 };
 
-DecodePlan decode_plan(const rcx_tensor& q, const rcx_tensor& k) {
+DecodePlan decode_plan(const rcx_tensor& q, const rcx_tensor& k, int ctas_per_sm = 2) {
   DecodePlan p;
   const int64_t B = q.shape[0], Hq = q.shape[2], Nk = k.shape[1], Hkv = std::max<int64_t>(k.shape[2], 1);
-  const int64_t want = std::max<int64_t>(1, (2 * (int64_t)sm_count() + Hkv * B - 1) / std::max<int64_t>(1, Hkv * B));
+  // at most one wave: splits x Hkv x B <= ctas_per_sm x SMs
+  const int64_t want = std::max<int64_t>(1, (ctas_per_sm * (int64_t)sm_count()) / std::max<int64_t>(1, Hkv * B));
   const int64_t cap = std::max<int64_t>(1, (Nk + 127) / 128);
   p.splits = (int)std::min<int64_t>(std::min<int64_t>(want, cap), 4096);
   p.keys_per_split = std::max<int64_t>(1, (Nk + p.splits - 1) / p.splits);
@@ -520,6 +522,120 @@ int decode_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, c
         default: attn_decode_kernel<8><<<grid, kDecThreads, 0, stream>>>(a); break;
       }
     }
+    if ((st = launch_status())) return st;
+  }
+  const int64_t threads = B * Hq * 32;
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 8));
+  LaunchScope scope(RCX_KERNEL_DECODE, stream);
+  if (o.dtype == RCX_BF16)
+    decode_combine_kernel<__nv_bfloat16><<<grid2, 256, 0, stream>>>(a);
+  else
+    decode_combine_kernel<float><<<grid2, 256, 0, stream>>>(a);
+  return launch_status();
+}
+
+// ------------------------------------------------------------ int8 KV cache
+
+// [B, N, H, d] int8 view: unit stride on d, non-negative strides.
+int check_i8(const rcx_tensor& t) {
+  for (int i = 0; i < 4; ++i)
+    if (t.shape[i] < 0) return RCX_ERR_INVALID_ARG;
+  if (t.dtype != RCX_I8) return RCX_ERR_INVALID_ARG;
+  const bool empty = t.shape[0] == 0 || t.shape[1] == 0 || t.shape[2] == 0 || t.shape[3] == 0;
+  if (!t.ptr && !empty) return RCX_ERR_INVALID_ARG;
+  if (t.stride[3] != 1 || t.stride[0] < 0 || t.stride[1] < 0 || t.stride[2] < 0) return RCX_ERR_INVALID_ARG;
+  return RCX_OK;
+}
+
+bool aligned_rows(const rcx_tensor& t, int bytes) {
+  const int per = bytes / elem_size(t.dtype);
+  return reinterpret_cast<uintptr_t>(t.ptr) % bytes == 0 && t.stride[0] % per == 0 && t.stride[1] % per == 0 &&
+         t.stride[2] % per == 0;
+}
+
+int quantize_i8_impl(const rcx_tensor& x, const rcx_tensor& c, float* scale, cudaStream_t stream) {
+  int st;
+  if ((st = check_act(x)) || (st = check_i8(c))) return st;
+  if (x.dtype != RCX_BF16) return RCX_ERR_UNSUPPORTED;
+  if (x.shape[3] != 128) return RCX_ERR_UNSUPPORTED;
+  for (int i = 0; i < 4; ++i)
+    if (c.shape[i] != x.shape[i]) return RCX_ERR_INVALID_ARG;
+  const int64_t rows = x.shape[0] * x.shape[1] * x.shape[2];
+  if (rows == 0) return RCX_OK;
+  if (!scale) return RCX_ERR_INVALID_ARG;
+  if (!aligned_rows(x, 8) || !aligned_rows(c, 4) || reinterpret_cast<uintptr_t>(scale) % 4) return RCX_ERR_ALIGNMENT;
+  QuantArgs a;
+  a.x = make_view(x);
+  a.c = make_view(c);
+  a.scale = scale;
+  a.rows = rows;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + 7) / 8, (int64_t)sm_count() * 8));
+  LaunchScope scope(RCX_KERNEL_DECODE, stream);
+  kv_quantize_int8_kernel<<<grid, 256, 0, stream>>>(a);
+  return launch_status();
+}
+
+int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scale, const rcx_tensor& v,
+                   const float* v_scale, const rcx_tensor& o, const rcx_tensor& lse, int64_t window, int64_t n_sink,
+                   double temperature, int64_t q_index, const int64_t* positions, int64_t n_positions,
+                   const double* inv_freq, int rope_flags, void* workspace, int64_t workspace_bytes,
+                   cudaStream_t stream) {
+  int st;
+  if ((st = check_act(q)) || (st = check_i8(k)) || (st = check_i8(v)) || (st = check_act(o))) return st;
+  const int64_t B = q.shape[0], Hq = q.shape[2], D = q.shape[3], Nk = k.shape[1], Hkv = k.shape[2];
+  if (q.shape[1] != 1 || o.shape[1] != 1) return RCX_ERR_INVALID_ARG;
+  if (q.dtype != RCX_BF16) return RCX_ERR_UNSUPPORTED;
+  if (D != 128 || k.shape[3] != 128 || v.shape[3] != 128 || o.shape[3] != 128) return RCX_ERR_UNSUPPORTED;
+  if (k.shape[0] != B || v.shape[0] != B || o.shape[0] != B || v.shape[1] != Nk || v.shape[2] != Hkv ||
+      o.shape[2] != Hq)
+    return RCX_ERR_INVALID_ARG;
+  if (Hkv <= 0 || Hq % Hkv) return RCX_ERR_INVALID_ARG;
+  const int64_t G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return RCX_ERR_UNSUPPORTED;
+  if (lse.ptr && (st = check_lse(lse, B, Hq, 1))) return st;
+  if (window < 0 || n_sink < 0 || q_index < 0) return RCX_ERR_INVALID_ARG;
+  if (!(temperature > 0.0) || !std::isfinite(temperature)) return RCX_ERR_INVALID_ARG;
+  if (rope_flags & ~RCX_ROTATE_Q) return rope_flags & RCX_ROTATE_K ? RCX_ERR_UNSUPPORTED : RCX_ERR_INVALID_ARG;
+  if (rope_flags && !inv_freq) return RCX_ERR_INVALID_ARG;
+  if (positions && n_positions <= std::max(q_index, Nk - 1)) return RCX_ERR_INVALID_ARG;
+  if (Nk > 0 && B > 0 && (!k_scale || !v_scale)) return RCX_ERR_INVALID_ARG;
+  // 16-byte code rows (cp.async), 8-byte q rows, 4-byte scales
+  if (!aligned_rows(q, 8) || !aligned_rows(k, 16) || !aligned_rows(v, 16) ||
+      !aligned_rows(o, o.dtype == RCX_BF16 ? 8 : 16))
+    return RCX_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(k_scale) % 4 || reinterpret_cast<uintptr_t>(v_scale) % 4) return RCX_ERR_ALIGNMENT;
+  if (B == 0 || Hq == 0) return RCX_OK;
+  if (B > 65535 || Hkv > 65535) return RCX_ERR_UNSUPPORTED;
+  const DecodePlan p = decode_plan(q, k, 3);
+  if (!workspace || workspace_bytes < p.total) return RCX_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return RCX_ERR_ALIGNMENT;
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = make_view(q); a.k = make_view(k); a.v = make_view(v); a.o = make_view(o);
+  a.lse = static_cast<float*>(lse.ptr);
+  a.lse_sb = lse.ptr ? lse.stride[0] : 0;
+  a.lse_sh = lse.ptr ? lse.stride[1] : 0;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.off_lse);
+  a.splits = p.splits;
+  a.keys_per_split = p.keys_per_split;
+  a.q_index = q_index;
+  a.window = window; a.n_sink = n_sink;
+  a.scale_log2 = (float)(1.4426950408889634074 / (std::sqrt((double)D) * temperature));
+  a.positions = positions;
+  a.rope_q = rope_flags & RCX_ROTATE_Q;
+  a.G = (int)G;
+  if (a.rope_q)
+    for (int i = 0; i < 64; ++i) a.f.theta[i] = inv_freq[i];
+  {
+    dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
+    LaunchScope scope(RCX_KERNEL_DECODE, stream);
+    auto kern = G == 1 ? attn_decode_i8_kernel<1>
+              : G == 2 ? attn_decode_i8_kernel<2>
+              : G == 4 ? attn_decode_i8_kernel<4>
+                       : attn_decode_i8_kernel<8>;
+    if (allow_smem(kern, kDqSmem)) return RCX_ERR_CUDA;
+    kern<<<grid, kDqWarps * 32, kDqSmem, stream>>>(a, k_scale, v_scale);
     if ((st = launch_status())) return st;
   }
   const int64_t threads = B * Hq * 32;
@@ -694,6 +810,23 @@ int rcx_attn_decode_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, 
                         int64_t workspace_bytes, void* stream) {
   return decode_impl(q, k, v, o, lse, window, n_sink, temperature, q_index, positions, n_positions, inv_freq,
                      rope_flags, workspace, workspace_bytes, as_stream(stream));
+}
+
+int rcx_kv_quantize_int8(rcx_tensor x, rcx_tensor codes, float* scale, void* stream) {
+  return quantize_i8_impl(x, codes, scale, as_stream(stream));
+}
+
+int64_t rcx_attn_decode_int8_workspace_size(rcx_tensor q, rcx_tensor k) {
+  if (check_act(q) || check_i8(k)) return -1;
+  return decode_plan(q, k, 3).total;
+}
+
+int rcx_attn_decode_int8_fwd(rcx_tensor q, rcx_tensor k, const float* k_scale, rcx_tensor v, const float* v_scale,
+                             rcx_tensor o, rcx_tensor lse, int64_t window, int64_t n_sink, double temperature,
+                             int64_t q_index, const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                             int rope_flags, void* workspace, int64_t workspace_bytes, void* stream) {
+  return decode_i8_impl(q, k, k_scale, v, v_scale, o, lse, window, n_sink, temperature, q_index, positions,
+                        n_positions, inv_freq, rope_flags, workspace, workspace_bytes, as_stream(stream));
 }
 
 int rcx_merge_partials(rcx_tensor o_a, rcx_tensor lse_a, rcx_tensor o_b, rcx_tensor lse_b, rcx_tensor o_out,

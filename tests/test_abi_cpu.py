@@ -96,3 +96,31 @@ def test_ring_workspace_size_is_deterministic(lib):
     # fp32 accumulator + its LSE + one shard's fp32 partial + its LSE (+ rotated K)
     assert n0 == N * Hq * D * 4 + Hq * N * 4 + 65536 * Hq * D * 4 + Hq * 65536 * 4
     assert n1 == n0 + N * Hkv * D * 2
+
+
+def test_int8_cache_argument_checks(lib):
+    """The int8 KV-cache entry points reject wrong dtypes and shapes before any launch."""
+    fake = 1 << 20   # never dereferenced: every case fails validation first
+    x = _host_tensor(fake, _lib.RCX_BF16, (1, 16, 2, 128), (4096, 256, 128, 1))
+    c8 = _host_tensor(fake, _lib.RCX_I8, (1, 16, 2, 128), (4096, 256, 128, 1))
+    c_bf = _host_tensor(fake, _lib.RCX_BF16, (1, 16, 2, 128), (4096, 256, 128, 1))
+    c_bad = _host_tensor(fake, _lib.RCX_I8, (1, 15, 2, 128), (4096, 256, 128, 1))
+    x32 = _host_tensor(fake, _lib.RCX_F32, (1, 16, 2, 128), (4096, 256, 128, 1))
+    x64 = _host_tensor(fake, _lib.RCX_BF16, (1, 16, 2, 64), (2048, 128, 64, 1))
+    sc = ctypes.c_void_p(fake)
+    assert lib.rcx_kv_quantize_int8(x, c_bf, sc, None) == _lib.RCX_ERR_INVALID_ARG    # codes not int8
+    assert lib.rcx_kv_quantize_int8(x, c_bad, sc, None) == _lib.RCX_ERR_INVALID_ARG   # shape mismatch
+    assert lib.rcx_kv_quantize_int8(x32, c8, sc, None) == _lib.RCX_ERR_UNSUPPORTED    # fp32 cache
+    assert lib.rcx_kv_quantize_int8(x64, c8, sc, None) == _lib.RCX_ERR_UNSUPPORTED    # d != 128
+    assert lib.rcx_kv_quantize_int8(x, c8, None, None) == _lib.RCX_ERR_INVALID_ARG    # no scale buffer
+    q = _host_tensor(fake, _lib.RCX_BF16, (1, 1, 8, 128), (1024, 1024, 128, 1))
+    null = _lib.RcxTensor()
+    assert lib.rcx_attn_decode_int8_workspace_size(q, c_bf) == -1                     # bf16 k
+    # bf16 cache passed to the int8 entry point, and int8 cache to the bf16 one
+    assert lib.rcx_attn_decode_int8_fwd(q, c_bf, sc, c_bf, sc, q, null, 0, 0, 1.0, 15, None, 0, None, 0, None, 0,
+                                        None) == _lib.RCX_ERR_INVALID_ARG
+    assert lib.rcx_attn_decode_fwd(q, c8, c8, q, null, 0, 0, 1.0, 15, None, 0, None, 0, None, 0,
+                                   None) == _lib.RCX_ERR_INVALID_ARG
+    # missing scales
+    assert lib.rcx_attn_decode_int8_fwd(q, c8, None, c8, sc, q, null, 0, 0, 1.0, 15, None, 0, None, 0, None, 0,
+                                        None) == _lib.RCX_ERR_INVALID_ARG
