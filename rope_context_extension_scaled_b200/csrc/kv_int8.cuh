@@ -56,9 +56,18 @@ __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const QuantArgs a
     for (int i = 0; i < kQRows; ++i) {
       const int64_t r = r0 + i * nwarps;
       const int64_t rr = r < a.rows ? r : r0;
-      const int64_t h = rr % a.x.H;
-      const int64_t n = (rr / a.x.H) % a.x.N;
-      const int64_t b = rr / (a.x.H * a.x.N);
+      int64_t h, n, b;
+      if (a.rows < (int64_t(1) << 31)) {          // 32-bit index arithmetic (the usual case)
+        const uint32_t r32 = (uint32_t)rr, H32 = (uint32_t)a.x.H, N32 = (uint32_t)a.x.N;
+        const uint32_t t32 = r32 / H32;
+        h = r32 - t32 * H32;
+        n = t32 % N32;
+        b = t32 / N32;
+      } else {
+        h = rr % a.x.H;
+        n = (rr / a.x.H) % a.x.N;
+        b = rr / (a.x.H * a.x.N);
+      }
       const __nv_bfloat16* xp = reinterpret_cast<const __nv_bfloat16*>(a.x.ptr) + b * a.x.sb + n * a.x.sn +
                                 h * a.x.sh + 4 * lane;
       u[i] = *reinterpret_cast<const uint2*>(xp);
