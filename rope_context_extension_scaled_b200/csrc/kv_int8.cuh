@@ -98,12 +98,13 @@ __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const QuantArgs a
 
 // ---------------------------------------------------------------- decode
 
-constexpr int kDqWarps = 4;
+constexpr int kDqWarps = 8;
 constexpr int kDqStages = 3;
 constexpr int kDqRow = 144;                                  // 128-byte code row + 16 pad (banks)
 constexpr int kDqTile = 16 * kDqRow;                         // one 16-key K or V tile
 constexpr int kDqStage = 2 * kDqTile + 2 * 64;               // K, V, 16 K scales, 16 V scales
-constexpr int kDqSmem = kDqWarps * kDqStages * kDqStage;     // 56,832 B: three CTAs per SM
+constexpr int kDqSmem = kDqWarps * kDqStages * kDqStage;     // 113,664 B: two CTAs (16 warps) per SM
+constexpr int kDqCtasPerSm = 2;
 static_assert(kDqSmem >= kDqWarps * kDecMaxG * 128 * 4, "merge area aliases the stage buffers");
 
 __device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {

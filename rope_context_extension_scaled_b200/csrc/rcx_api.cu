@@ -606,7 +606,7 @@ int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scal
   if (reinterpret_cast<uintptr_t>(k_scale) % 4 || reinterpret_cast<uintptr_t>(v_scale) % 4) return RCX_ERR_ALIGNMENT;
   if (B == 0 || Hq == 0) return RCX_OK;
   if (B > 65535 || Hkv > 65535) return RCX_ERR_UNSUPPORTED;
-  const DecodePlan p = decode_plan(q, k, 3);
+  const DecodePlan p = decode_plan(q, k, kDqCtasPerSm);
   if (!workspace || workspace_bytes < p.total) return RCX_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return RCX_ERR_ALIGNMENT;
   DecodeArgs a;
@@ -818,7 +818,7 @@ int rcx_kv_quantize_int8(rcx_tensor x, rcx_tensor codes, float* scale, void* str
 
 int64_t rcx_attn_decode_int8_workspace_size(rcx_tensor q, rcx_tensor k) {
   if (check_act(q) || check_i8(k)) return -1;
-  return decode_plan(q, k, 3).total;
+  return decode_plan(q, k, kDqCtasPerSm).total;
 }
 
 int rcx_attn_decode_int8_fwd(rcx_tensor q, rcx_tensor k, const float* k_scale, rcx_tensor v, const float* v_scale,
