@@ -20,8 +20,7 @@ source pages (cited per function as "page title, section"):
   * kwkr.cn long-context article, section 2.2: ring attention pseudo-code
     (roll the KV chunks by one each step, aggregate online).
 
-Readings taken where the pages are silent, garbled or disagree (each is also
-listed in DESIGN.md):
+Readings taken where the pages are silent, garbled or disagree:
   * rotation pairs are adjacent dimensions (2i, 2i+1), rotated counter-clockwise
     by phi = m * theta_i;
   * NTK-by-parts band edges are L_train/beta (short wavelengths, unscaled) and
@@ -32,7 +31,9 @@ listed in DESIGN.md):
   * logits are scaled by 1/(sqrt(d) * t);
   * partial results are combined by an LSE-weighted merge (the page's plain
     "output += block_output" is only right after that weighting);
-  * the ring visits, at step t, KV block (r - t) mod P on shard r.
+  * the ring visits, at step t, KV block (r - t) mod P on shard r;
+  * an int8 KV cache is symmetric per row of d values: scale = amax / 127 and
+    code = rint(x * 127 / amax), decided in IEEE fp32.
 
 Parity pins for every function live in tests/test_oracle_pins.py.
 """
