@@ -36,11 +36,10 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "causal attention fwd TFLOP/s and % of B200 BF16 tensor peak at 128K and 1M"
-# DRAM bytes (read + write) per attention launch, from a one-pass ncu capture of
-# every attention launch of one step of the same command (summary and command in
-# profiles/attn_tc_traffic_llama3_70b_1m_ring.md).  Valid for the attention
-# kernel as captured; re-take it when the kernel changes.
-ATTN_TRAFFIC_PER_LAUNCH = {"llama3_70b_1m_ring": 3.729e9}
+# DRAM bytes (read + write) per attention launch of the named workload, from an
+# ncu capture of the attention kernel as currently built (empty until one is
+# taken; reported as roofline.traffic).
+ATTN_TRAFFIC_PER_LAUNCH = {}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

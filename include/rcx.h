@@ -166,6 +166,30 @@ int rcx_attn_blockwise_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
                            const double* inv_freq, int rope_flags, void* stream);
 
 /*
+ * rcx_attn_blockwise_merge_fwd -- one step of the Ring-Attention loop: the
+ * attention of rcx_attn_blockwise_fwd over this call's keys, merged in the
+ * kernel's epilogue into a previous partial result over other keys by the
+ * rule of rcx_merge_partials ("Context window extension: 4K to 1M" 5.3,
+ * "output += block_output" made exact by the LSE weights; kwkr.cn 2.2,
+ * online aggregation).  No partial buffer is written and no merge pass runs.
+ *
+ * acc: fp32 [B, Nq, Hq, d], the previous partial's normalised O, 16-byte
+ * aligned base and token/head/batch strides that are multiples of 4
+ * elements; acc_lse: its [B, Hq, Nq, 1] natural-log LSE (-inf marks a row
+ * with no keys so far).  o, lse: the merged result (o f32 or bf16); o may be
+ * acc itself and lse may be acc_lse (in-place accumulation: keep lse non-NULL
+ * until the last step, or the accumulator's LSE is not updated).  Every other
+ * argument, the mask and the paths are as rcx_attn_blockwise_fwd.  A row
+ * with no visible key in either partial gets O = 0 and lse = -inf.
+ */
+int rcx_attn_blockwise_merge_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o,
+                                 rcx_tensor lse, rcx_tensor acc, rcx_tensor acc_lse,
+                                 int64_t kv_block, int64_t window, int64_t n_sink,
+                                 double temperature, int64_t q_start, int64_t k_start,
+                                 const int64_t* positions, int64_t n_positions,
+                                 const double* inv_freq, int rope_flags, void* stream);
+
+/*
  * rcx_attn_decode_fwd -- attention of one new query token per (batch, head)
  * against a KV cache ("Context Extension" concept page, KV-cache section:
  * each generated token computes Q, K, V, appends K, V to the cache and
@@ -285,9 +309,11 @@ int rcx_ring_attn_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rc
  * message on stderr) before anything is launched.  The call itself makes no
  * cudaMalloc/cudaFree and calls no allocating library routine.
  *
- * The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (the device current at that moment) and keeps it;
- * make that first call on a device before any stream capture.
+ * Every call looks up the array's device address on the current device with
+ * cudaGetSymbolAddress (a host-side query: no allocation, no synchronisation),
+ * so the address stays right if the device's context is torn down and
+ * re-created.  The first call on a device may load the library's device code
+ * there; make that first call before any stream capture.
  * Every call uses the same array and leaves its last contents there; nothing
  * in it has to start at zero, because each call writes every scratch byte it
  * reads.  Calls whose work overlaps on the GPU (different streams, or
@@ -304,7 +330,10 @@ int rcx_ring_attn_fwd_noalloc(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tens
  * same as rcx_ring_attn_fwd but q, k, v, o (and lse if non-NULL) are HOST
  * buffers (pinned for full copy speed); the call allocates the device copies
  * and workspace, copies in, computes, copies out and frees, synchronously on
- * `stream`.  positions is a HOST array here.
+ * `stream`.  positions is a HOST array here.  Because the call synchronises,
+ * it also reads (and clears) the device status words: a bounded wait that ran
+ * out in one of its kernels returns RCX_ERR_DEVICE_TIMEOUT (o and lse then
+ * hold incomplete results).
  */
 int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
                            int64_t kv_block, int64_t window, int64_t n_sink, double temperature,

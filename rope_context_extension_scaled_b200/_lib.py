@@ -32,7 +32,7 @@ EXPORTS = (
     "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
     "rcx_ring_attn_fwd_noalloc", "rcx_rope_freqs_per_pair", "rcx_attn_decode_workspace_size",
     "rcx_attn_decode_fwd", "rcx_kv_quantize_int8", "rcx_attn_decode_int8_workspace_size",
-    "rcx_attn_decode_int8_fwd",
+    "rcx_attn_decode_int8_fwd", "rcx_attn_blockwise_merge_fwd",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20   # RCX_NOALLOC_SCRATCH_BYTES in include/rcx.h
 KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3, "decode": 4}
@@ -82,6 +82,9 @@ def load():
     lib.rcx_attn_decode_int8_fwd.restype = ctypes.c_int
     lib.rcx_attn_blockwise_fwd.argtypes = [T, T, T, T, T, i64, i64, i64, f64, i64, i64, vp, i64, pd,
                                            ctypes.c_int, vp]
+    lib.rcx_attn_blockwise_merge_fwd.argtypes = [T, T, T, T, T, T, T, i64, i64, i64, f64, i64, i64, vp, i64, pd,
+                                                 ctypes.c_int, vp]
+    lib.rcx_attn_blockwise_merge_fwd.restype = ctypes.c_int
     lib.rcx_merge_partials.argtypes = [T, T, T, T, T, T, vp]
     lib.rcx_ring_workspace_size.argtypes = [T, T, i64, ctypes.c_int]
     lib.rcx_ring_workspace_size.restype = i64
@@ -222,6 +225,20 @@ def attn_blockwise_fwd(q, k, v, o=None, lse=None, kv_block=0, window=0, n_sink=0
                                        int(window), int(n_sink), float(temperature), int(q_start), int(k_start),
                                        pp, npos, fp, int(rope_flags), _stream(q.device))
     _check(st, "rcx_attn_blockwise_fwd")
+    return o, lse
+
+
+def attn_blockwise_merge_fwd(q, k, v, o, lse, acc, acc_lse, kv_block=0, window=0, n_sink=0, temperature=1.0,
+                             q_start=0, k_start=0, positions=None, inv_freq=None, rope_flags=0):
+    """Attention over this call's keys merged into the partial (acc, acc_lse)
+    in the kernel's epilogue; o / lse may be acc / acc_lse (in place)."""
+    arr, fp = _freq_ptr(inv_freq)
+    pp, npos = _pos(positions)
+    st = load().rcx_attn_blockwise_merge_fwd(view(q), view(k), view(v), view(o), lse_view(lse), view(acc),
+                                             lse_view(acc_lse), int(kv_block), int(window), int(n_sink),
+                                             float(temperature), int(q_start), int(k_start), pp, npos, fp,
+                                             int(rope_flags), _stream(q.device))
+    _check(st, "rcx_attn_blockwise_merge_fwd")
     return o, lse
 
 

@@ -17,6 +17,13 @@ struct AttnArgs {
   int rope_flags;             // RCX_ROTATE_Q | RCX_ROTATE_K
   int pairs;                  // d / 2
   int G;                      // Hq / Hkv
+  // Optional previous partial result over other keys (a ring accumulator):
+  // acc.ptr == nullptr: none.  Otherwise fp32 [B, Nq, Hq, d] (normalised O)
+  // and its natural-log LSE [B, Hq, Nq]; the kernel merges its own result
+  // into it by the LSE rule before writing o and lse (which may alias acc).
+  View4 acc;
+  const float* acc_lse;
+  int64_t acc_lse_sb, acc_lse_sh;
   Freqs f;
 };
 

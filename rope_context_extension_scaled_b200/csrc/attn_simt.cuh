@@ -138,14 +138,35 @@ __global__ void __launch_bounds__(kSimtBR * TPR) attn_simt_kernel(const AttnArgs
     }
   }
 
+  // Epilogue: O = ca * O_prev + cb * acc with cb = 1 / l alone, or the LSE
+  // merge with a previous partial result (ring accumulator) when one is given.
+  const float lse_b = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  float cb = l > 0.f ? 1.f / l : 0.f, ca = 0.f, lse_out = lse_b;
+  const float* accp = nullptr;
+  if (a.acc.ptr != nullptr && row_ok) {
+    accp = reinterpret_cast<const float*>(a.acc.ptr) + b * a.acc.sb + (r0 + row) * a.acc.sn + h * a.acc.sh;
+    const float lse_a = a.acc_lse[b * a.acc_lse_sb + h * a.acc_lse_sh + r0 + row];
+    const float mm = fmaxf(lse_a, lse_b);
+    if (mm == -INFINITY) {
+      cb = 0.f;
+      lse_out = -INFINITY;
+    } else {
+      const float wa = expf(lse_a - mm), wb = expf(lse_b - mm), den = wa + wb;
+      ca = wa / den;
+      cb *= wb / den;
+      lse_out = mm + logf(den);
+    }
+  }
+  __syncwarp();   // every part of the row has read the previous LSE before it is overwritten
   if (row_ok) {
-    const float inv = l > 0.f ? 1.f / l : 0.f;
     Tout* op = reinterpret_cast<Tout*>(a.o.ptr) + b * a.o.sb + (r0 + row) * a.o.sn + h * a.o.sh;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) op[e * TPR + part] = from_f<Tout>(acc[e] * inv);
-    if (a.lse && part == 0)
-      a.lse[b * a.lse_sb + h * a.lse_sh + r0 + row] =
-          l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    for (int e = 0; e < 32; ++e) {
+      float x = acc[e] * cb;
+      if (accp) x = fmaf(ca, accp[e * TPR + part], x);
+      op[e * TPR + part] = from_f<Tout>(x);
+    }
+    if (a.lse && part == 0) a.lse[b * a.lse_sb + h * a.lse_sh + r0 + row] = lse_out;
   }
 }
 

@@ -638,42 +638,69 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_OFINAL + s), 0, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        // O = ca * O_prev + cb * O_unnormalised: cb = 1 / l alone, or the LSE
+        // merge with a previous partial over other keys (ring accumulator):
+        // weights w = exp(lse - max) of both partials.
+        const float lse_b = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        float cb = l > 0.f ? 1.f / l : 0.f, ca = 0.f, lse_out = lse_b;
+        const float* accp = nullptr;
+        if (a.acc.ptr != nullptr && row_ok) {
+          accp = reinterpret_cast<const float*>(a.acc.ptr) + bb * a.acc.sb + row * a.acc.sn + head[s] * a.acc.sh;
+          const float lse_a = a.acc_lse[bb * a.acc_lse_sb + head[s] * a.acc_lse_sh + row];
+          const float mm = fmaxf(lse_a, lse_b);
+          if (mm == -INFINITY) {
+            cb = 0.f;
+            lse_out = -INFINITY;
+          } else {
+            const float wa = expf(lse_a - mm), wb = expf(lse_b - mm), den = wa + wb;
+            ca = wa / den;
+            cb *= wb / den;
+            lse_out = mm + logf(den);
+          }
+        }
         Tout* op = reinterpret_cast<Tout*>(a.o.ptr) + bb * a.o.sb + row * a.o.sn + head[s] * a.o.sh;
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cbk = 0; cbk < 4; ++cbk) {
           uint32_t o[32];
           if (n_tiles > 0) {
-            tmem_ld32(tO[s] + lane_off + cb * 32, o);
+            tmem_ld32(tO[s] + lane_off + cbk * 32, o);
             tmem_wait_ld();
           } else {
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = 0u;
           }
           if (row_ok) {
+            float f[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(o[c]) * cb;
+            if (accp) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 4) {
+                const float4 pv = *reinterpret_cast<const float4*>(accp + cbk * 32 + c);
+                f[c] = fmaf(ca, pv.x, f[c]);
+                f[c + 1] = fmaf(ca, pv.y, f[c + 1]);
+                f[c + 2] = fmaf(ca, pv.z, f[c + 2]);
+                f[c + 3] = fmaf(ca, pv.w, f[c + 3]);
+              }
+            }
             if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
               for (int c = 0; c < 32; c += 8) {
                 uint4 v;
-                v.x = f2_to_bf2(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
-                v.y = f2_to_bf2(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-                v.z = f2_to_bf2(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
-                v.w = f2_to_bf2(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
-                *reinterpret_cast<uint4*>(op + cb * 32 + c) = v;
+                v.x = f2_to_bf2(f[c + 0], f[c + 1]);
+                v.y = f2_to_bf2(f[c + 2], f[c + 3]);
+                v.z = f2_to_bf2(f[c + 4], f[c + 5]);
+                v.w = f2_to_bf2(f[c + 6], f[c + 7]);
+                *reinterpret_cast<uint4*>(op + cbk * 32 + c) = v;
               }
             } else {
 #pragma unroll
-              for (int c = 0; c < 32; c += 4) {
-                float4 v = make_float4(__uint_as_float(o[c]) * inv, __uint_as_float(o[c + 1]) * inv,
-                                       __uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-                *reinterpret_cast<float4*>(op + cb * 32 + c) = v;
-              }
+              for (int c = 0; c < 32; c += 4)
+                *reinterpret_cast<float4*>(op + cbk * 32 + c) = make_float4(f[c], f[c + 1], f[c + 2], f[c + 3]);
             }
           }
         }
-        if (row_ok && a.lse)
-          a.lse[bb * a.lse_sb + head[s] * a.lse_sh + row] =
-              l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        if (row_ok && a.lse) a.lse[bb * a.lse_sb + head[s] * a.lse_sh + row] = lse_out;
       }
     }
   }
@@ -683,92 +710,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, 512);
-}
-
-// ------------------------------------------------------------------ host side
-
-static std::atomic<int64_t> g_tc_inject_spins{0};
-inline void attn_tc_set_inject(int64_t spins) { g_tc_inject_spins.store(spins); }
-
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  // looked up once, thread-safely
-  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
-  }();
-  return fn;
-}
-
-// 4-D map over a [B, N, H, 128] bf16 view, box = 64 columns x 1 head x 128 tokens.
-static int make_tile_map(CUtensorMap* map, const rcx_tensor& t) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return RCX_ERR_CUDA;
-  const int64_t B = t.shape[0], N = t.shape[1], H = t.shape[2], D = t.shape[3];
-  // Unit-size dimensions get a dense stride (TMA wants 16-byte multiples).
-  const int64_t sh = H > 1 ? t.stride[2] : D;
-  const int64_t sn = N > 1 ? t.stride[1] : sh * H;
-  const int64_t sb = B > 1 ? t.stride[0] : sn * N;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(sn * 2), (cuuint64_t)(sb * 2)};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)kTcBM, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t.ptr, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? RCX_OK : RCX_ERR_CUDA;
-}
-
-static bool tc_view_ok(const rcx_tensor& t) {
-  if (t.dtype != RCX_BF16 || t.shape[3] != kTcD) return false;
-  if (reinterpret_cast<uintptr_t>(t.ptr) % 16) return false;
-  for (int i = 0; i < 3; ++i)
-    if (t.stride[i] % 8) return false;
-  if (t.shape[1] > 0x7fffffff - 2 * kTcBM || t.shape[2] > 0x7fffffff || t.shape[0] > 0x7fffffff) return false;
-  return true;
-}
-
-template <typename ScopeFn>
-static int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v,
-                          const rcx_tensor& o, cudaStream_t stream, ScopeFn&& scope_fn) {
-  if (!tc_view_ok(q) || !tc_view_ok(k) || !tc_view_ok(v)) return RCX_ERR_ALIGNMENT;
-  const int oes = o.dtype == RCX_BF16 ? 2 : 4;
-  if (reinterpret_cast<uintptr_t>(o.ptr) % 16 || o.stride[0] % (16 / oes) || o.stride[1] % (16 / oes) ||
-      o.stride[2] % (16 / oes))
-    return RCX_ERR_ALIGNMENT;
-  if (a.k.N == 0) {
-    // no keys at all: every row is empty -> handled by the kernel (zero tiles)
-  }
-  CUtensorMap mq, mk, mv;
-  int st;
-  if ((st = make_tile_map(&mq, q)) || (st = make_tile_map(&mk, k)) || (st = make_tile_map(&mv, v))) return st;
-  TcParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.a = a;
-  p.pair_heads = (a.G % 2 == 0) ? 1 : 0;
-  const int64_t rows_per_item = p.pair_heads ? kTcBM : 2 * kTcBM;
-  p.n_rb = (int)((a.q.N + rows_per_item - 1) / rows_per_item);
-  p.n_hg = (int)(p.pair_heads ? a.q.H / 2 : a.q.H);
-  p.inject_spins = g_tc_inject_spins.load();
-  const int64_t items = (int64_t)p.n_rb * p.n_hg * a.q.B;
-  if (items <= 0) return RCX_OK;
-  if (items > 0x7fffffff) return RCX_ERR_UNSUPPORTED;
-  const cudaError_t ea = o.dtype == RCX_BF16
-                             ? cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal)
-                             : cudaFuncSetAttribute(attn_tc_kernel<float>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal);
-  if (ea != cudaSuccess) return RCX_ERR_CUDA;
-  auto scope = scope_fn(stream);
-  if (o.dtype == RCX_BF16)
-    attn_tc_kernel<__nv_bfloat16><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
-  else
-    attn_tc_kernel<float><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? RCX_OK : RCX_ERR_CUDA;
 }
 
 }  // namespace rcx

@@ -66,11 +66,32 @@ template <> __device__ __forceinline__ float from_f<float>(float x) { return x; 
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 // Device status word (RCX_OK or the first RCX_ERR_DEVICE_TIMEOUT recorded).
-// The library is one translation unit, so a file-scope definition suffices.
-__device__ int g_device_status = 0;
+// The kernels are compiled in several translation units without relocatable
+// device code, so each unit that includes this header has its own word;
+// device_status_exchange() reads and clears the word of the calling unit.
+static __device__ int g_device_status = 0;
 
 __device__ __forceinline__ void record_device_error(int code) {
   atomicCAS(&g_device_status, 0, code);
+}
+
+// Reads this translation unit's status word into *status and clears it,
+// ordered on `stream` (synchronises the stream).
+static inline int device_status_exchange(cudaStream_t stream, int* status) {
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) !=
+      cudaSuccess)
+    return RCX_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return RCX_ERR_CUDA;
+  *status = v;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess)
+      return RCX_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return RCX_ERR_CUDA;
+  }
+  return RCX_OK;
 }
 
 }  // namespace rcx

@@ -45,7 +45,7 @@ struct QuantArgs {
 // per pass (grid-strided) and issues all their loads before any arithmetic.
 constexpr int kQRows = 4;
 
-__global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const QuantArgs a) {
+static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
   const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;

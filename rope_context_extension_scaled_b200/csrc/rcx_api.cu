@@ -11,12 +11,12 @@
 #include <mutex>
 #include <vector>
 
+#include "launch.h"
 #include "common.cuh"
 #include "rope_apply.cuh"
 #include "merge.cuh"
 #include "attn_common.cuh"
 #include "attn_simt.cuh"
-#include "attn_tc.cuh"
 #include "attn_decode.cuh"
 #include "kv_int8.cuh"
 #include "rope_freqs.inc"
@@ -24,8 +24,6 @@
 using namespace rcx;
 
 namespace {
-
-// ------------------------------------------------------------ launch accounting
 
 struct Stats {
   std::mutex mu;
@@ -51,32 +49,55 @@ Stats& stats() {
   return *s;
 }
 
-// Counts a launch of `kind`; with timing on, records events around it.
-class LaunchScope {
- public:
-  LaunchScope(int kind, cudaStream_t stream) : kind_(kind), stream_(stream) {
-    Stats& st = stats();
-    std::lock_guard<std::mutex> g(st.mu);
-    ++st.launches[kind];
-    if (st.timing) {
-      start_ = st.take();
-      stop_ = st.take();
-      cudaEventRecord(start_, stream_);
-    }
-  }
-  ~LaunchScope() {
-    if (!start_) return;
-    cudaEventRecord(stop_, stream_);
-    Stats& st = stats();
-    std::lock_guard<std::mutex> g(st.mu);
-    st.spans[kind_].push_back({start_, stop_});
-  }
+}  // namespace
 
- private:
-  int kind_;
-  cudaStream_t stream_;
-  cudaEvent_t start_ = nullptr, stop_ = nullptr;
-};
+// ------------------------------------------------------------ launch accounting
+
+namespace rcx {
+
+LaunchScope::LaunchScope(int kind, cudaStream_t stream) : kind_(kind), stream_(stream) {
+  Stats& st = stats();
+  std::lock_guard<std::mutex> g(st.mu);
+  ++st.launches[kind];
+  if (st.timing) {
+    start_ = st.take();
+    stop_ = st.take();
+    cudaEventRecord(start_, stream_);
+  }
+}
+
+LaunchScope::~LaunchScope() {
+  if (!start_) return;
+  cudaEventRecord(stop_, stream_);
+  Stats& st = stats();
+  std::lock_guard<std::mutex> g(st.mu);
+  st.spans[kind_].push_back({start_, stop_});
+}
+
+int sm_count() {
+  // initialised once, thread-safely (every device this library targets is a B200)
+  static const int n = [] {
+    int dev = 0, c = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+      c = 148;
+    return c;
+  }();
+  return n;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "librcx: launch failed: %s\n", cudaGetErrorString(e));
+    return RCX_ERR_CUDA;
+  }
+  return RCX_OK;
+}
+
+}  // namespace rcx
+
+namespace {
 
 constexpr int kAbiVersion = 100;
 
@@ -122,34 +143,6 @@ int check_lse(const rcx_tensor& t, int64_t B, int64_t H, int64_t N) {
   return RCX_OK;
 }
 
-int sm_count() {
-  // initialised once, thread-safely (every device this library targets is a B200)
-  static const int n = [] {
-    int dev = 0, c = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
-      c = 148;
-    return c;
-  }();
-  return n;
-}
-
-// Opt a kernel into more than 48 KB of dynamic shared memory.
-template <typename K>
-int allow_smem(K kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess
-             ? RCX_OK
-             : RCX_ERR_CUDA;
-}
-
-int launch_status() {
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    std::fprintf(stderr, "librcx: launch failed: %s\n", cudaGetErrorString(e));
-    return RCX_ERR_CUDA;
-  }
-  return RCX_OK;
-}
 
 rcx_tensor null_tensor() {
   rcx_tensor t;
@@ -233,8 +226,7 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
         all_dense = all_dense && dense(*ins[i]) && dense(*outs[i]) && tb <= kRopeBulkBytes && tb % 16 == 0;
       }
     if (all_dense) {
-      const size_t smem = (size_t)kRopeBulkStages * kRopeBulkBytes + kRopeMaxAngles * sizeof(float2) +
-                          kRopeBulkStages * sizeof(uint64_t);
+      const size_t smem = kRopeBulkSmem;
       for (int i = 0; i < 2; ++i) {
         if (!ins[i]->ptr) continue;
         RopeBulkArgs b;
@@ -248,19 +240,13 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
         b.pairs = (int)(D / 2);
         b.token_bytes = ins[i]->shape[2] * D * elem_size(dtype);
         b.tok_per_chunk = (int)std::max<int64_t>(
-            1, std::min<int64_t>(kRopeBulkBytes / b.token_bytes, (kRopeMaxAngles / 2) / b.pairs));
+            1, std::min<int64_t>(kRopeBulkBytes / b.token_bytes, kRopeBulkTab / b.pairs));
+        b.row_chunks = (int)(b.token_bytes / 16);
+        b.d_chunks = (int)(D * elem_size(dtype) / 16);
         for (int j = 0; j < b.pairs; ++j) b.f.theta[j] = inv_freq[j];
         const int64_t chunks = (b.n_tok + b.tok_per_chunk - 1) / b.tok_per_chunk;
         const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 2);
-        LaunchScope scope(RCX_KERNEL_ROPE, stream);
-        if (dtype == RCX_BF16) {
-          if (allow_smem(rope_bulk_kernel<__nv_bfloat16>, smem)) return RCX_ERR_CUDA;
-          rope_bulk_kernel<__nv_bfloat16><<<grid, kRopeThreads, smem, stream>>>(b);
-        } else {
-          if (allow_smem(rope_bulk_kernel<float>, smem)) return RCX_ERR_CUDA;
-          rope_bulk_kernel<float><<<grid, kRopeThreads, smem, stream>>>(b);
-        }
-        const int st = launch_status();
+        const int st = rope_bulk_launch(b, dtype, grid, smem, stream);
         if (st) return st;
       }
       return RCX_OK;
@@ -305,15 +291,7 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 6);
   auto same = [](const View4& x, const View4& y) { return x.sb == y.sb && x.sn == y.sn && x.sh == y.sh; };
   const bool same_layout = (!has_q || same(a.q_in, a.q_out)) && (!has_k || same(a.k_in, a.k_out));
-  LaunchScope scope(RCX_KERNEL_ROPE, stream);
-  if (dtype == RCX_BF16) {
-    if (same_layout) rope_apply_kernel<__nv_bfloat16, true><<<grid, kRopeThreads, 0, stream>>>(a);
-    else rope_apply_kernel<__nv_bfloat16, false><<<grid, kRopeThreads, 0, stream>>>(a);
-  } else {
-    if (same_layout) rope_apply_kernel<float, true><<<grid, kRopeThreads, 0, stream>>>(a);
-    else rope_apply_kernel<float, false><<<grid, kRopeThreads, 0, stream>>>(a);
-  }
-  return launch_status();
+  return rope_apply_launch(a, dtype, same_layout, grid, stream);
 }
 
 // ---------------------------------------------------------------------- merge
@@ -349,40 +327,19 @@ int merge_impl(const rcx_tensor& oa, const rcx_tensor& la, const rcx_tensor& ob,
   a.d4 = (int)(D / 4);
   const int64_t warps = B * N;     // one warp per token at a time
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8));
-  LaunchScope scope(RCX_KERNEL_MERGE, stream);
-  if (oo.dtype == RCX_BF16)
-    merge_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
-  else
-    merge_kernel<float><<<grid, 256, 0, stream>>>(a);
-  return launch_status();
+  return merge_launch(a, oo.dtype, grid, stream);
 }
 
 // ------------------------------------------------------------------ attention
 
-template <typename T, typename Tout>
-int launch_simt(const AttnArgs& a, cudaStream_t stream) {
-  const int64_t D = a.q.D;
-  const int64_t tiles = (a.q.N + kSimtBR - 1) / kSimtBR;
-  dim3 grid((unsigned)tiles, (unsigned)a.q.H, (unsigned)a.q.B);
-  const size_t smem = (size_t)2 * kSimtBC * D * sizeof(float);
-  LaunchScope scope(RCX_KERNEL_ATTN_SIMT, stream);
-  if (D == 32) {
-    if (allow_smem(attn_simt_kernel<T, Tout, 1>, smem)) return RCX_ERR_CUDA;
-    attn_simt_kernel<T, Tout, 1><<<grid, kSimtBR * 1, smem, stream>>>(a);
-  } else if (D == 64) {
-    if (allow_smem(attn_simt_kernel<T, Tout, 2>, smem)) return RCX_ERR_CUDA;
-    attn_simt_kernel<T, Tout, 2><<<grid, kSimtBR * 2, smem, stream>>>(a);
-  } else {
-    if (allow_smem(attn_simt_kernel<T, Tout, 4>, smem)) return RCX_ERR_CUDA;
-    attn_simt_kernel<T, Tout, 4><<<grid, kSimtBR * 4, smem, stream>>>(a);
-  }
-  return launch_status();
-}
-
+// acc / acc_lse: optional previous partial result over other keys (fp32
+// normalised O and its LSE), merged into this call's result in the epilogue;
+// o / lse may alias them.  Null pointers: no previous partial.
 int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, const rcx_tensor& o,
               const rcx_tensor& lse, int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
               int64_t q_start, int64_t k_start, const int64_t* positions, int64_t n_positions,
-              const double* inv_freq, int rope_flags, cudaStream_t stream) {
+              const double* inv_freq, int rope_flags, cudaStream_t stream, const rcx_tensor* acc = nullptr,
+              const rcx_tensor* acc_lse = nullptr) {
   int st;
   if ((st = check_act(q)) || (st = check_act(k)) || (st = check_act(v)) || (st = check_act(o))) return st;
   const int64_t B = q.shape[0], Nq = q.shape[1], Hq = q.shape[2], D = q.shape[3];
@@ -399,6 +356,15 @@ int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
   if (rope_flags && !inv_freq) return RCX_ERR_INVALID_ARG;
   if (rope_flags && positions && n_positions < std::max(q_start + Nq, k_start + Nk)) return RCX_ERR_INVALID_ARG;
   if (D < 2 || (D & 1)) return RCX_ERR_INVALID_ARG;
+  const bool merging = acc != nullptr && acc->ptr != nullptr;
+  if (merging) {
+    if ((st = check_act(*acc))) return st;
+    if (acc->dtype != RCX_F32) return RCX_ERR_INVALID_ARG;
+    for (int j = 0; j < 4; ++j)
+      if (acc->shape[j] != o.shape[j]) return RCX_ERR_INVALID_ARG;
+    if (!acc_lse || (st = check_lse(*acc_lse, B, Hq, Nq))) return st ? st : RCX_ERR_INVALID_ARG;
+    if (!vec16_ok(*acc)) return RCX_ERR_ALIGNMENT;
+  }
   if (B == 0 || Nq == 0) return RCX_OK;
 
   AttnArgs a;
@@ -415,6 +381,12 @@ int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
   a.rope_flags = rope_flags;
   a.pairs = (int)(D / 2);
   a.G = (int)(Hq / Hkv);
+  if (merging) {
+    a.acc = make_view(*acc);
+    a.acc_lse = static_cast<const float*>(acc_lse->ptr);
+    a.acc_lse_sb = acc_lse->stride[0];
+    a.acc_lse_sh = acc_lse->stride[1];
+  }
   if (rope_flags) {
     if (a.pairs > kMaxPairs) return RCX_ERR_INVALID_ARG;
     for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
@@ -422,13 +394,12 @@ int attn_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
 
   if (q.dtype == RCX_BF16 && D == 128) {
     if (rope_flags & RCX_ROTATE_K) return RCX_ERR_UNSUPPORTED;
-    return attn_tc_launch(a, q, k, v, o, stream, [&](cudaStream_t s) { return LaunchScope(RCX_KERNEL_ATTN_TC, s); });
+    return attn_tc_launch(a, q, k, v, o, stream);
   }
   if (D != 32 && D != 64 && D != 128) return RCX_ERR_UNSUPPORTED;
   if (q.dtype == RCX_F32)
-    return o.dtype == RCX_F32 ? launch_simt<float, float>(a, stream) : launch_simt<float, __nv_bfloat16>(a, stream);
-  return o.dtype == RCX_F32 ? launch_simt<__nv_bfloat16, float>(a, stream)
-                            : launch_simt<__nv_bfloat16, __nv_bfloat16>(a, stream);
+    return o.dtype == RCX_F32 ? attn_simt_launch_f32_f32(a, stream) : attn_simt_launch_f32_bf16(a, stream);
+  return o.dtype == RCX_F32 ? attn_simt_launch_bf16_f32(a, stream) : attn_simt_launch_bf16_bf16(a, stream);
 }
 
 // --------------------------------------------------------------------- decode
@@ -505,33 +476,11 @@ int decode_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, c
     for (int i = 0; i < 64; ++i) a.f.theta[i] = inv_freq[i];
   {
     dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
-    LaunchScope scope(RCX_KERNEL_DECODE, stream);
-    if (al(k, 16) && al(v, 16)) {
-      // tensor-core form: 16-byte rows of k and v for cp.async
-      auto kern = G == 1 ? attn_decode_mma_kernel<1>
-                : G == 2 ? attn_decode_mma_kernel<2>
-                : G == 4 ? attn_decode_mma_kernel<4>
-                         : attn_decode_mma_kernel<8>;
-      if (allow_smem(kern, kDmSmem)) return RCX_ERR_CUDA;
-      kern<<<grid, kDmWarps * 32, kDmSmem, stream>>>(a);
-    } else {
-      switch (G) {
-        case 1: attn_decode_kernel<1><<<grid, kDecThreads, 0, stream>>>(a); break;
-        case 2: attn_decode_kernel<2><<<grid, kDecThreads, 0, stream>>>(a); break;
-        case 4: attn_decode_kernel<4><<<grid, kDecThreads, 0, stream>>>(a); break;
-        default: attn_decode_kernel<8><<<grid, kDecThreads, 0, stream>>>(a); break;
-      }
-    }
-    if ((st = launch_status())) return st;
+    if ((st = decode_launch(a, (int)G, al(k, 16) && al(v, 16), grid, stream))) return st;
   }
   const int64_t threads = B * Hq * 32;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 8));
-  LaunchScope scope(RCX_KERNEL_DECODE, stream);
-  if (o.dtype == RCX_BF16)
-    decode_combine_kernel<__nv_bfloat16><<<grid2, 256, 0, stream>>>(a);
-  else
-    decode_combine_kernel<float><<<grid2, 256, 0, stream>>>(a);
-  return launch_status();
+  return decode_combine_launch(a, o.dtype, grid2, stream);
 }
 
 // ------------------------------------------------------------ int8 KV cache
@@ -570,9 +519,7 @@ int quantize_i8_impl(const rcx_tensor& x, const rcx_tensor& c, float* scale, cud
   a.scale = scale;
   a.rows = rows;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + 7) / 8, (int64_t)sm_count() * 8));
-  LaunchScope scope(RCX_KERNEL_DECODE, stream);
-  kv_quantize_int8_kernel<<<grid, 256, 0, stream>>>(a);
-  return launch_status();
+  return quantize_i8_launch(a, grid, stream);
 }
 
 int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scale, const rcx_tensor& v,
@@ -629,23 +576,23 @@ int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scal
     for (int i = 0; i < 64; ++i) a.f.theta[i] = inv_freq[i];
   {
     dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
-    LaunchScope scope(RCX_KERNEL_DECODE, stream);
-    auto kern = G == 1 ? attn_decode_i8_kernel<1>
-              : G == 2 ? attn_decode_i8_kernel<2>
-              : G == 4 ? attn_decode_i8_kernel<4>
-                       : attn_decode_i8_kernel<8>;
-    if (allow_smem(kern, kDqSmem)) return RCX_ERR_CUDA;
-    kern<<<grid, kDqWarps * 32, kDqSmem, stream>>>(a, k_scale, v_scale);
-    if ((st = launch_status())) return st;
+    if ((st = decode_i8_launch(a, (int)G, k_scale, v_scale, grid, stream))) return st;
   }
   const int64_t threads = B * Hq * 32;
   const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 8));
-  LaunchScope scope(RCX_KERNEL_DECODE, stream);
-  if (o.dtype == RCX_BF16)
-    decode_combine_kernel<__nv_bfloat16><<<grid2, 256, 0, stream>>>(a);
-  else
-    decode_combine_kernel<float><<<grid2, 256, 0, stream>>>(a);
-  return launch_status();
+  return decode_combine_launch(a, o.dtype, grid2, stream);
+}
+
+// -------------------------------------------------------------- device status
+
+// Reads and clears the status words of every kernel family with bounded
+// waits (synchronising `s`); the tensor-core attention's word wins if both are set.
+int device_status_all(cudaStream_t s, int* out) {
+  int a = 0, b = 0, st;
+  if ((st = status_exchange_attn_tc(s, &a))) return st;
+  if ((st = status_exchange_rope(s, &b))) return st;
+  *out = a != 0 ? a : b;
+  return RCX_OK;
 }
 
 // ----------------------------------------------------------------------- ring
@@ -653,7 +600,7 @@ int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scal
 struct RingPlan {
   int64_t B, N, Hq, Hkv, D, kv, P;
   bool rotate_k_separately;
-  int64_t off_acc, off_lacc, off_part, off_lpart, off_krot, total;
+  int64_t off_acc, off_lacc, off_krot, total;
 };
 
 RingPlan ring_plan(const rcx_tensor& q, const rcx_tensor& k, int64_t kv_block, int rope_flags) {
@@ -665,8 +612,6 @@ RingPlan ring_plan(const rcx_tensor& q, const rcx_tensor& k, int64_t kv_block, i
   int64_t off = 0;
   p.off_acc = off;   off = align256(off + p.B * p.N * p.Hq * p.D * 4);
   p.off_lacc = off;  off = align256(off + p.B * p.Hq * p.N * 4);
-  p.off_part = off;  off = align256(off + p.B * p.kv * p.Hq * p.D * 4);
-  p.off_lpart = off; off = align256(off + p.B * p.Hq * p.kv * 4);
   p.off_krot = off;
   if (p.rotate_k_separately) off = align256(off + p.B * p.N * p.Hkv * p.D * 2);
   p.total = off;
@@ -688,8 +633,6 @@ int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
   char* ws = static_cast<char*>(workspace);
   rcx_tensor acc = make_tensor(ws + p.off_acc, RCX_F32, p.B, p.N, p.Hq, p.D);
   rcx_tensor lacc = make_lse(ws + p.off_lacc, p.B, p.Hq, p.N);
-  rcx_tensor part = make_tensor(ws + p.off_part, RCX_F32, p.B, p.kv, p.Hq, p.D);
-  rcx_tensor lpart = make_lse(ws + p.off_lpart, p.B, p.Hq, p.kv);
 
   rcx_tensor kk = k;
   int flags = rope_flags;
@@ -734,22 +677,16 @@ int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
       }
       rcx_tensor as = token_slice(acc, i0, ni);
       rcx_tensor las = lse_slice(lacc, i0, ni);
-      if (t == first[r]) {
+      if (t == first[r]) {          // first visible block: the fp32 accumulator
         st = attn_impl(qs, ks, vs, as, las, 0, window, n_sink, temperature, i0, j0, positions, n_positions,
                        inv_freq, flags, stream);
-        if (st) return st;
-        continue;
-      }
-      rcx_tensor ps = token_slice(part, 0, ni);
-      rcx_tensor lps = lse_slice(lpart, 0, ni);
-      st = attn_impl(qs, ks, vs, ps, lps, 0, window, n_sink, temperature, i0, j0, positions, n_positions,
-                     inv_freq, flags, stream);
-      if (st) return st;
-      if (t == last[r]) {
+      } else if (t == last[r]) {    // last: merged with the accumulator into the final output
         rcx_tensor lo = lse.ptr ? ls_final : las;
-        st = merge_impl(as, las, ps, lps, os_final, lo, stream);
-      } else {
-        st = merge_impl(as, las, ps, lps, null_tensor(), null_tensor(), stream);
+        st = attn_impl(qs, ks, vs, os_final, lo, 0, window, n_sink, temperature, i0, j0, positions, n_positions,
+                       inv_freq, flags, stream, &as, &las);
+      } else {                      // merged into the accumulator in place
+        st = attn_impl(qs, ks, vs, as, las, 0, window, n_sink, temperature, i0, j0, positions, n_positions,
+                       inv_freq, flags, stream, &as, &las);
       }
       if (st) return st;
     }
@@ -797,6 +734,17 @@ int rcx_attn_blockwise_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
                            const double* inv_freq, int rope_flags, void* stream) {
   return attn_impl(q, k, v, o, lse, kv_block, window, n_sink, temperature, q_start, k_start, positions,
                    n_positions, inv_freq, rope_flags, as_stream(stream));
+}
+
+int rcx_attn_blockwise_merge_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
+                                 rcx_tensor acc, rcx_tensor acc_lse, int64_t kv_block, int64_t window,
+                                 int64_t n_sink, double temperature, int64_t q_start, int64_t k_start,
+                                 const int64_t* positions, int64_t n_positions, const double* inv_freq,
+                                 int rope_flags, void* stream) {
+  const bool empty = q.shape[0] == 0 || q.shape[1] == 0 || q.shape[2] == 0 || q.shape[3] == 0;
+  if (!acc.ptr && !empty) return RCX_ERR_INVALID_ARG;
+  return attn_impl(q, k, v, o, lse, kv_block, window, n_sink, temperature, q_start, k_start, positions,
+                   n_positions, inv_freq, rope_flags, as_stream(stream), &acc, &acc_lse);
 }
 
 int64_t rcx_attn_decode_workspace_size(rcx_tensor q, rcx_tensor k) {
@@ -892,6 +840,12 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
     st = RCX_ERR_CUDA;
   cudaFreeAsync(dev, s);
   if (cudaStreamSynchronize(s) != cudaSuccess && !st) st = RCX_ERR_CUDA;
+  // This call is synchronous, so a bounded wait that ran out in one of its
+  // kernels is reported here (and the status word cleared), not left for a
+  // later rcx_device_status().
+  int dev_st = RCX_OK;
+  if (!st && device_status_all(s, &dev_st) != RCX_OK) st = RCX_ERR_CUDA;
+  if (!st && dev_st != RCX_OK) st = dev_st;
   return st;
 }
 
@@ -901,32 +855,26 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
 
 // Scratch of rcx_ring_attn_fwd_noalloc: a module-scope device array, so the
 // entry point needs no cudaMalloc.  In host code this name only stands for
-// the array; its device address comes from cudaGetSymbolAddress, once per
-// device, with that device current.
+// the array; its device address comes from cudaGetSymbolAddress with the
+// device of the call current.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RCX_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kNoAllocMaxDevices] = {};
-
+// Device address of the scratch array on the current device.  Looked up on
+// every call rather than cached: the lookup is a host-side query (no
+// allocation, no synchronisation), and a cached address would go stale if the
+// device's context were torn down and re-created (cudaDeviceReset reloads the
+// module, and the array may then sit elsewhere).
 int noalloc_scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return RCX_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return RCX_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> g(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) {
-      std::fprintf(stderr, "librcx: cudaGetSymbolAddress of the no-alloc scratch failed: %s\n",
-                   cudaGetErrorString(e));
-      return RCX_ERR_CUDA;
-    }
-    g_noalloc_addr[dev] = p;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
+    std::fprintf(stderr, "librcx: cudaGetSymbolAddress of the no-alloc scratch failed: %s\n",
+                 cudaGetErrorString(e));
+    return RCX_ERR_CUDA;
   }
-  *out = g_noalloc_addr[dev];
+  *out = p;
   return RCX_OK;
 }
 
@@ -955,17 +903,7 @@ int rcx_ring_attn_fwd_noalloc(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tens
 
 int rcx_device_status(void* stream, int* status_out) {
   if (!status_out) return RCX_ERR_INVALID_ARG;
-  cudaStream_t s = as_stream(stream);
-  int v = 0;
-  if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return RCX_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return RCX_ERR_CUDA;
-  *status_out = v;
-  const int zero = 0;
-  if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return RCX_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return RCX_ERR_CUDA;
-  return RCX_OK;
+  return device_status_all(as_stream(stream), status_out);
 }
 
 int rcx_stats_enable_timing(int on) {

@@ -163,19 +163,29 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_apply_kernel(const RopeA
 }
 
 // ---------------------------------------------------------------------------
-// Bulk-copy path for dense layouts ([B, N, H, d] with no gaps, in and out).
-// A token's H x d values are one contiguous row, so a chunk of T tokens is one
-// contiguous span: cp.async.bulk brings it into shared memory (four stages per
-// CTA, three loading while one is rotated; two CTAs per SM).  Two warps build
-// the next chunk's T x d/2 (cos, sin) table (with consecutive positions: one
-// precise angle per pair and the angle-addition identity for the rest) while
-// six warps rotate the current chunk on its way out with coalesced 16-byte
-// stores.  Every wait on a copy is bounded (about
-// one second) and
-// records RCX_ERR_DEVICE_TIMEOUT if it runs out.
+// Path for dense layouts ([B, N, H, d] with no gaps, in and out): a token's
+// H x d values are one contiguous row, so a chunk of T consecutive tokens is
+// one contiguous span of T * token_bytes bytes.  A CTA takes chunks in turn;
+// each thread owns the same kRopePieces 16-byte pieces of every chunk (piece
+// e = thread + 256 k), so which token and which pairs a piece holds is decoded
+// once.  The next chunk's pieces are loaded into registers before the current
+// one is rotated and stored, so every thread keeps 2 x kRopePieces 16-byte
+// loads in flight; one barrier per chunk publishes the chunk's angles.
+//
+// Angles with consecutive positions (positions == NULL; position = token
+// index within its batch entry): cos/sin of (n0 + t) theta come from the
+// angle-addition identity applied once to two exact values, the chunk's base
+// angle n0 theta (one precise angle per pair per chunk) and the step angle
+// t theta (t < T, a table built once per CTA).  Both come from rope_cos_sin,
+// so the applied angle is within a few 1e-7 rad of m theta and there is no
+// recurrence whose rounding grows with t.  With explicit positions every
+// (token, pair) angle of the chunk is computed directly into a table; a chunk
+// that crosses into the next batch entry computes its angles per piece.
 
-constexpr int kRopeBulkStages = 4;
-constexpr int kRopeBulkBytes = 18432;      // bytes of one stage (T * token bytes)
+constexpr int kRopePieces = 8;                         // 16-byte pieces per thread per chunk
+constexpr int kRopeBulkBytes = kRopeThreads * kRopePieces * 16;   // 32 KB chunk
+constexpr int kRopeBulkTab = kRopeMaxAngles / 2;       // float2 entries of one angle table (>= T * pairs)
+constexpr size_t kRopeBulkSmem = 3 * kRopeBulkTab * sizeof(float2);
 
 struct RopeBulkArgs {
   const void* in;
@@ -187,160 +197,137 @@ struct RopeBulkArgs {
   int tok_per_chunk;           // T
   int pairs;                   // d / 2
   int d;
+  int row_chunks;              // 16-byte pieces per token (token_bytes / 16)
+  int d_chunks;                // 16-byte pieces per head (d * element size / 16)
   Freqs f;
 };
 
-__device__ __forceinline__ uint32_t rb_smem(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ bool rb_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok = 0;
-  uint64_t t0 = 0;
-  for (uint32_t it = 0;; ++it) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    if (it == 0) t0 = t;
-    else if (t - t0 > 1000000000ull) {
-      record_device_error(RCX_ERR_DEVICE_TIMEOUT);
-      return false;
-    }
-  }
+// cos/sin product (a then b): the angle-addition identity.
+__device__ __forceinline__ float2 cs_add(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBulkArgs a) {
-  // Warps 0-5 rotate chunk i while warps 6-7 build the angle table of chunk
-  // i + 1 into the other table buffer; one barrier per chunk.
   constexpr int kElems = 16 / sizeof(T);
   constexpr int kPairsPerChunk = kElems / 2;
-  constexpr int kRotThreads = kRopeThreads - 64;
-  extern __shared__ __align__(128) uint8_t rb_raw[];
-  uint8_t* stage_buf = rb_raw;                                                        // [stages][kRopeBulkBytes]
-  float2* cs = reinterpret_cast<float2*>(rb_raw + kRopeBulkStages * kRopeBulkBytes);  // [2][kRopeMaxAngles / 2]
-  uint64_t* full = reinterpret_cast<uint64_t*>(cs + kRopeMaxAngles);                  // [stages]
-  __shared__ int abort_flag;
-  constexpr int kTab = kRopeMaxAngles / 2;
+  extern __shared__ __align__(16) float2 rb_tabs[];     // [3][kRopeBulkTab]
+  const int tid = threadIdx.x;
+  const int pairs = a.pairs;
+  const bool dense_pos = a.positions == nullptr;
+  // dense positions: tabs[0] = step table [T][pairs], tabs[1] = base angles [2][pairs];
+  // explicit positions: tabs[1], tabs[2] = direct tables [T][pairs] (double buffer)
+  float2* step_tab = rb_tabs;
+  float2* base_tab = rb_tabs + kRopeBulkTab;
+  auto direct_tab = [&](int buf) { return rb_tabs + (1 + buf) * kRopeBulkTab; };
 
   const int64_t n_chunks = (a.n_tok + a.tok_per_chunk - 1) / a.tok_per_chunk;
-  const int64_t first = blockIdx.x, step = gridDim.x;
-  const bool rot = threadIdx.x < kRotThreads;
+  const int64_t step = gridDim.x;
   auto chunk_tokens = [&](int64_t c) {
     const int64_t left = a.n_tok - c * a.tok_per_chunk;
     return (int)(left < a.tok_per_chunk ? left : a.tok_per_chunk);
   };
-  auto issue_load = [&](int64_t c, int st) {
+  // First token n0 (within its batch entry) of chunk c; true when the chunk
+  // stays in one batch entry.
+  auto in_one_entry = [&](int64_t c, int64_t& n0) {
     const int64_t t0 = c * a.tok_per_chunk;
-    const uint32_t bytes = (uint32_t)(chunk_tokens(c) * a.token_bytes);
-    const uint32_t bar = rb_smem(&full[st]);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            rb_smem(stage_buf + st * kRopeBulkBytes)),
-        "l"(static_cast<const uint8_t*>(a.in) + t0 * a.token_bytes), "r"(bytes), "r"(bar)
-        : "memory");
+    n0 = t0 - (t0 / a.N) * a.N;
+    return n0 + chunk_tokens(c) <= a.N;
   };
-  // Angle table of chunk c into cs[buf]: one precise angle per pair and the
-  // angle-addition identity for consecutive positions, else direct angles.
-  auto build_table = [&](int64_t c, int buf) {
-    const int lt = threadIdx.x - kRotThreads;          // 0 .. 63
+  // Angles chunk c needs, into buffer `buf`.  Threads 0, 4, 8, ... take the
+  // base angles, so the extra sincos work spreads over all warps.
+  auto prepare = [&](int64_t c, int buf) {
+    int64_t n0;
+    const bool one = in_one_entry(c, n0);
+    if (dense_pos) {
+      if (one)
+        for (int j = tid; j < 4 * pairs; j += kRopeThreads)
+          if ((j & 3) == 0) {
+            float cc, sn;
+            rope_cos_sin(n0, a.f.theta[j >> 2], cc, sn);
+            base_tab[buf * kMaxPairs + (j >> 2)] = make_float2(cc, sn);
+          }
+      return;
+    }
     const int ntok = chunk_tokens(c);
-    const int64_t t0 = c * a.tok_per_chunk;
-    const int64_t n0 = t0 - (t0 / a.N) * a.N;
-    float2* tab = cs + buf * kTab;
-    if (!a.positions && n0 + ntok <= a.N) {
-      for (int p = lt; p < a.pairs; p += 64) {
-        float cc, sn, c1, s1;
-        rope_cos_sin(n0, a.f.theta[p], cc, sn);
-        rope_cos_sin(1, a.f.theta[p], c1, s1);
-        tab[p] = make_float2(cc, sn);
-        for (int t = 1; t < ntok; ++t) {
-          const float c2 = cc * c1 - sn * s1, s2 = sn * c1 + cc * s1;
-          cc = c2;
-          sn = s2;
-          tab[t * a.pairs + p] = make_float2(cc, sn);
-        }
-      }
-    } else {
-      for (int e = lt; e < ntok * a.pairs; e += 64) {
-        const int t = e / a.pairs, p = e - t * a.pairs;
-        int64_t n = n0 + t;
-        while (n >= a.N) n -= a.N;
-        const int64_t m = a.positions ? a.positions[n] : n;
-        float cc, sn;
-        rope_cos_sin(m, a.f.theta[p], cc, sn);
-        tab[t * a.pairs + p] = make_float2(cc, sn);
-      }
+    float2* tab = direct_tab(buf);
+    for (int e = tid; e < ntok * pairs; e += kRopeThreads) {
+      const int t = e / pairs, p = e - t * pairs;
+      int64_t n = n0 + t;
+      while (n >= a.N) n -= a.N;
+      float cc, sn;
+      rope_cos_sin(a.positions[n], a.f.theta[p], cc, sn);
+      tab[t * pairs + p] = make_float2(cc, sn);
     }
   };
 
-  if (threadIdx.x == 0) {
-    abort_flag = 0;
-    for (int st = 0; st < kRopeBulkStages; ++st)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(rb_smem(&full[st])) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int st = 0; st < kRopeBulkStages; ++st)
-      if (first + st * step < n_chunks) issue_load(first + st * step, st);
+  // This thread's pieces: token and first pair of piece e = tid + 256 k.
+  int pt[kRopePieces], pp[kRopePieces];
+#pragma unroll
+  for (int k = 0; k < kRopePieces; ++k) {
+    const int e = tid + k * kRopeThreads;
+    pt[k] = e / a.row_chunks;
+    pp[k] = ((e - pt[k] * a.row_chunks) % a.d_chunks) * kPairsPerChunk;
   }
-  if (!rot && first < n_chunks) build_table(first, 0);
-  __syncthreads();
+  auto load = [&](int64_t c, uint4* u) {
+    const int total = chunk_tokens(c) * a.row_chunks;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.in) +
+                                                      c * a.tok_per_chunk * a.token_bytes);
+#pragma unroll
+    for (int k = 0; k < kRopePieces; ++k) {
+      const int e = tid + k * kRopeThreads;
+      if (e < total) u[k] = src[e];
+    }
+  };
 
-  int i = 0;
-  for (int64_t c = first; c < n_chunks; c += step, ++i) {
-    const int st = i % kRopeBulkStages;
+  if (dense_pos)
+    for (int e = tid; e < a.tok_per_chunk * pairs; e += kRopeThreads) {
+      const int t = e / pairs, p = e - t * pairs;
+      float cc, sn;
+      rope_cos_sin(t, a.f.theta[p], cc, sn);
+      step_tab[e] = make_float2(cc, sn);
+    }
+  int64_t c = blockIdx.x;
+  if (c < n_chunks) prepare(c, 0);
+  uint4 u[kRopePieces], un[kRopePieces];
+  if (c < n_chunks) load(c, u);
+  for (int i = 0; c < n_chunks; c += step, ++i) {
     const int buf = i & 1;
-    if (rot) {
-      if (!rb_wait(rb_smem(&full[st]), (i / kRopeBulkStages) & 1)) abort_flag = 1;
-      if (!abort_flag) {
-        const int ntok = chunk_tokens(c);
-        const int64_t t0 = c * a.tok_per_chunk;
-        const uint8_t* src = stage_buf + st * kRopeBulkBytes;
-        uint8_t* dst = static_cast<uint8_t*>(a.out) + t0 * a.token_bytes;
-        const float2* tab = cs + buf * kTab;
-        const int row_chunks = (int)(a.token_bytes / 16);
-        const int d_chunks = a.d / kElems;
-        for (int e = threadIdx.x; e < ntok * row_chunks; e += kRotThreads) {
-          const int t = e / row_chunks, rc = e - t * row_chunks;
-          const int dc = rc % d_chunks;                  // 16-byte chunk within the head
-          uint4 u = *reinterpret_cast<const uint4*>(src + (size_t)e * 16);
-          rope_chunk_regs<T>(u, &tab[t * a.pairs + dc * kPairsPerChunk]);
-          *reinterpret_cast<uint4*>(dst + (size_t)e * 16) = u;
+    __syncthreads();                                  // angles of chunk c are in buffer buf
+    const bool more = c + step < n_chunks;
+    if (more) load(c + step, un);                     // next chunk's loads in flight during this one
+    int64_t n0;
+    const bool one = in_one_entry(c, n0);
+    const int total = chunk_tokens(c) * a.row_chunks;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + c * a.tok_per_chunk * a.token_bytes);
+    const float2* base = base_tab + buf * kMaxPairs;
+    const float2* dtab = direct_tab(buf);
+#pragma unroll
+    for (int k = 0; k < kRopePieces; ++k) {
+      const int e = tid + k * kRopeThreads;
+      if (e < total) {
+        float2 cs[kPairsPerChunk];
+        const int t = pt[k], p0 = pp[k];
+        if (dense_pos && one) {
+#pragma unroll
+          for (int q = 0; q < kPairsPerChunk; ++q) cs[q] = cs_add(base[p0 + q], step_tab[t * pairs + p0 + q]);
+        } else if (!dense_pos) {
+#pragma unroll
+          for (int q = 0; q < kPairsPerChunk; ++q) cs[q] = dtab[t * pairs + p0 + q];
+        } else {
+          int64_t n = n0 + t;
+          while (n >= a.N) n -= a.N;
+#pragma unroll
+          for (int q = 0; q < kPairsPerChunk; ++q) rope_cos_sin(n, a.f.theta[p0 + q], cs[q].x, cs[q].y);
         }
+        rope_chunk_regs<T>(u[k], cs);
+        dst[e] = u[k];
       }
-    } else if (c + step < n_chunks) {
-      build_table(c + step, buf ^ 1);
     }
-    __syncthreads();
-    if (abort_flag) break;
-    if (threadIdx.x == 0) {
-      const int64_t nc = c + (int64_t)kRopeBulkStages * step;
-      if (nc < n_chunks) issue_load(nc, st);
-    }
-  }
-  if (threadIdx.x == 0 && abort_flag) {
-    // let copies that may still be landing finish before the CTA exits
-    for (int st = 0; st < kRopeBulkStages; ++st) {
-      uint32_t ok;
-      uint64_t t0, t;
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-      do {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(rb_smem(&full[st])), "r"(0u)
-            : "memory");
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      } while (!ok && t - t0 < 100000000ull);
+    if (more) {
+      prepare(c + step, buf ^ 1);
+#pragma unroll
+      for (int k = 0; k < kRopePieces; ++k) u[k] = un[k];
     }
   }
 }

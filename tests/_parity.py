@@ -8,6 +8,7 @@ import numpy as np
 import torch
 
 from oracle import rcx_oracle as orc
+from rope_context_extension_scaled_b200 import _lib
 
 # Tolerances.  The bf16 path rounds the rotated Q and K to bf16 (u = 2^-8)
 # before the tensor-core product: a logit q.k / sqrt(d) with |q|, |k| ~ sqrt(d)
@@ -19,6 +20,16 @@ TOL_F32_MAX = 1e-4
 TOL_BF16_O_MAX = 2e-2
 TOL_BF16_O_MEAN = 2e-3
 TOL_BF16_LSE_MEAN = 1e-3
+
+
+def schedule(scheme, base, d, L_train, L_target, alpha=1.0, beta=32.0):
+    """One RoPE schedule evaluated by both sides: (inv, t) from the library,
+    handed to the GPU call, and (oinv, ot) from the oracle, used for the
+    expected values, so an end-to-end comparison also checks the library's
+    frequencies and temperature."""
+    inv, t = _lib.rope_freqs(scheme, base, d, L_train, L_target, alpha, beta)
+    oinv, ot = orc.rope_freqs(scheme, base, d, L_train, L_target, alpha, beta)
+    return inv, t, oinv, ot
 
 
 def np64(t):

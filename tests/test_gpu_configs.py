@@ -13,7 +13,7 @@ from rope_context_extension_scaled_b200 import _lib
 from rope_context_extension_scaled_b200.configs import ORDER, WORKLOADS
 from rope_context_extension_scaled_b200.inputs import make_qkv, sample_rows
 from rope_context_extension_scaled_b200.runner import run_workload
-from tests._parity import all_rows, assert_bf16, assert_f32, errors, gather_gpu, oracle_rows
+from tests._parity import schedule, all_rows, assert_bf16, assert_f32, errors, gather_gpu, oracle_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -36,11 +36,11 @@ def test_workload_parity(name):
     run = run_workload(w, q, k, v)
     o, lse = run()
     torch.cuda.synchronize()
-    inv, t = _lib.rope_freqs(w.scheme, w.base, w.d, w.L_train, w.L_target, w.alpha, w.beta)
+    inv, t, oinv, ot = schedule(w.scheme, w.base, w.d, w.L_train, w.L_target, w.alpha, w.beta)
     rows = all_rows(w.N, w.Hq) if not w.sample_rows else sample_rows(w.N, w.Hq, w.sample_rows, seed=0,
                                                                        must_tokens=_must_tokens(w))
     assert sum(len(r) for r in rows.values()) >= min(4096, w.N * w.Hq)
-    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, w.window, w.n_sink)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], oinv, ot, rows, w.window, w.n_sink)
     err = errors(*gather_gpu(o, lse, rows), Or, Lr)
     print(name, err)
     (assert_f32 if w.dtype == "f32" else assert_bf16)(err)

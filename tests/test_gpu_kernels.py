@@ -12,7 +12,7 @@ import torch
 from oracle import rcx_oracle as orc
 from rope_context_extension_scaled_b200 import _lib
 from rope_context_extension_scaled_b200.inputs import make_qkv
-from tests._parity import (all_rows, assert_bf16, assert_f32, errors, gather_gpu, np64, oracle_rows)
+from tests._parity import (schedule, all_rows, assert_bf16, assert_f32, errors, gather_gpu, np64, oracle_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -26,7 +26,7 @@ DEV = "cuda"
 @pytest.mark.parametrize("pos_kind", ["arange", "random"])
 def test_rope_apply_matches_oracle(dtype, N, Hq, Hkv, d, pos_kind):
     q, k, _ = make_qkv(2, N, Hq, Hkv, d, dtype, seed=1, device=DEV)
-    inv, _ = _lib.rope_freqs(_lib.NTK, 5e5, d, 8192, 8192 * 128)
+    inv, _, oinv, _ = schedule(_lib.NTK, 5e5, d, 8192, 8192 * 128)
     pos = None
     p_np = np.arange(N)
     if pos_kind == "random":
@@ -39,7 +39,7 @@ def test_rope_apply_matches_oracle(dtype, N, Hq, Hkv, d, pos_kind):
     torch.cuda.synchronize()
     for x, y in ((q, qo), (k, ko)):
         for b in range(2):
-            ref = orc.rope_rotate(np64(x[b]), p_np, inv)
+            ref = orc.rope_rotate(np64(x[b]), p_np, oinv)
             got = np64(y[b])
             if dtype == torch.float32:
                 assert np.abs(got - ref).max() < 1e-5
@@ -49,7 +49,7 @@ def test_rope_apply_matches_oracle(dtype, N, Hq, Hkv, d, pos_kind):
 
 def test_rope_apply_in_place_equals_out_of_place():
     q, k, _ = make_qkv(1, 257, 4, 2, 128, torch.bfloat16, seed=2, device=DEV)
-    inv, _ = _lib.rope_freqs(_lib.YARN, 1e4, 128, 4096, 32768)
+    inv, _, oinv, _ = schedule(_lib.YARN, 1e4, 128, 4096, 32768)
     qo, ko = torch.empty_like(q), torch.empty_like(k)
     _lib.rope_apply(q, k, inv, q_out=qo, k_out=ko)
     q2, k2 = q.clone(), k.clone()
@@ -66,7 +66,7 @@ def test_rope_angle_error_at_one_million():
     # Unit vectors (1, 0) in every pair, rotated in fp32: the applied angle
     # must be within 1e-5 rad of m * theta' (exact, 60-digit arithmetic).
     d = 128
-    inv, _ = _lib.rope_freqs(_lib.NTK, 5e5, d, 8192, 1 << 20)
+    inv, _, oinv, _ = schedule(_lib.NTK, 5e5, d, 8192, 1 << 20)
     ms = [0, 1, 65535, 999_999, 1_048_575, (1 << 24) - 1]
     x = torch.zeros(1, len(ms), 1, d, dtype=torch.float32, device=DEV)
     x[..., 0::2] = 1.0
@@ -86,9 +86,42 @@ def test_rope_angle_error_at_one_million():
     assert worst <= 2e-6, worst      # observed: fp32 sincos of the fp64-reduced angle
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_rope_bulk_path_angle_error_near_one_million(d):
+    # Dense layout and positions == NULL take the bulk-copy kernel, whose
+    # angles for consecutive tokens come from an exact per-chunk base angle
+    # and an exact step angle (angle-addition identity).  Unit vectors (1, 0)
+    # in every pair, fp32, N = 2^20 tokens of one head (chunks of 16 tokens at
+    # d = 128, 32 at d = 64): the applied angle of every pair must be within
+    # 1e-5 rad of m * theta' (60-digit arithmetic), including chunks that start
+    # just below m = 1,048,575 and every offset within a chunk.
+    N = 1 << 20
+    inv, _, _, _ = schedule(_lib.NTK, 5e5, d, 8192, 1 << 20)
+    x = torch.zeros(1, N, 1, d, dtype=torch.float32, device=DEV)
+    x[..., 0::2] = 1.0
+    _lib.rope_apply(x, None, inv)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(7)
+    toks = np.unique(np.concatenate([np.arange(N - 192, N), np.arange(0, 40),
+                                     rng.integers(0, N, size=96)]))
+    out = x[0, torch.as_tensor(toks, device=DEV), 0].cpu().numpy().astype(np.float64)
+    got = np.arctan2(out[:, 1::2], out[:, 0::2])
+    mpmath.mp.dps = 40
+    two_pi = 2 * mpmath.pi
+    worst = 0.0
+    for r, m in enumerate(toks):
+        for i in range(d // 2):
+            e = mpmath.mpf(int(m)) * mpmath.mpf(float(inv[i]))
+            ex = float(e - two_pi * mpmath.nint(e / two_pi))
+            diff = abs((got[r, i] - ex + math.pi) % (2 * math.pi) - math.pi)
+            worst = max(worst, diff)
+    print(f"bulk rope_apply d={d}: worst angle error {worst:.3e} rad over {len(toks)} tokens")
+    assert worst <= 1e-5, worst
+
+
 def test_rope_apply_rejects_misaligned():
     q = torch.zeros(1, 4, 1, 130, dtype=torch.bfloat16, device=DEV)[..., 1:129]   # 2-byte offset
-    inv, _ = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    inv, _, oinv, _ = schedule(_lib.PLAIN, 1e4, 128, 10, 10)
     with pytest.raises(_lib.RcxError) as e:
         _lib.rope_apply(q, None, inv)
     assert e.value.status == _lib.RCX_ERR_ALIGNMENT
@@ -106,11 +139,11 @@ def _run_attn(q, k, v, inv, t, rows=None, **kw):
     (512, 64, 0, 0), (200, 0, 0, 0), (333, 50, 40, 3), (97, 7, 0, 0), (130, 0, 16, 0)])
 def test_fp32_attention_fused_rope(N, kv_block, window, n_sink):
     q, k, v = make_qkv(1, N, 2, 1, 64, torch.float32, seed=4, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.PI, 1e4, 64, 256, 512)
+    inv, t, oinv, ot = schedule(_lib.PI, 1e4, 64, 256, 512)
     o, lse = _run_attn(q, k, v, inv, t, kv_block=kv_block, window=window, n_sink=n_sink,
                        rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
     rows = all_rows(N, 2)
-    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, window, n_sink)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], oinv, ot, rows, window, n_sink)
     assert_f32(errors(*gather_gpu(o, lse, rows), Or, Lr))
 
 
@@ -118,12 +151,12 @@ def test_fp32_attention_fused_rope(N, kv_block, window, n_sink):
                                       (640, 4, 4), (257, 6, 3)])
 def test_bf16_tensor_core_attention(N, Hq, Hkv):
     q, k, v = make_qkv(1, N, Hq, Hkv, 128, torch.bfloat16, seed=5, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 8192, 32768)
+    inv, t, oinv, ot = schedule(_lib.NTK, 5e5, 128, 8192, 32768)
     krot = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, k_out=krot)
     o, lse = _run_attn(q, krot, v, inv, t, rope_flags=_lib.ROTATE_Q)
     rows = all_rows(N, Hq)
-    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], oinv, ot, rows)
     assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
 
 
@@ -132,13 +165,13 @@ def test_bf16_tensor_core_attention(N, Hq, Hkv):
 def test_bf16_window_sinks_ring_order(window, n_sink, kv_block):
     N = 777
     q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=6, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.YARN, 1e4, 128, 256, 2048)
+    inv, t, oinv, ot = schedule(_lib.YARN, 1e4, 128, 256, 2048)
     krot = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, k_out=krot)
     o, lse = _run_attn(q, krot, v, inv, t, rope_flags=_lib.ROTATE_Q, window=window, n_sink=n_sink,
                        kv_block=kv_block)
     rows = all_rows(N, 4)
-    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, window, n_sink)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], oinv, ot, rows, window, n_sink)
     assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
 
 
@@ -150,14 +183,14 @@ def test_bf16_offsets_positions_and_fp32_output():
     g = torch.Generator(device=DEV)
     g.manual_seed(9)
     pos = torch.randint(0, 1 << 20, (Nk,), generator=g, device=DEV, dtype=torch.int64)
-    inv, t = _lib.rope_freqs(_lib.DYN_NTK, 5e5, 128, 8192, 131072)
+    inv, t, oinv, ot = schedule(_lib.DYN_NTK, 5e5, 128, 8192, 131072)
     krot = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, positions=pos, k_out=krot)
     o, lse = _run_attn(q, krot, v, inv, t, rope_flags=_lib.ROTATE_Q, q_start=500, k_start=0, positions=pos,
                        out_dtype=torch.float32)
     assert o.dtype == torch.float32
     rows = all_rows(Nq, 4)
-    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, positions=pos, q_start=500, k_start=0)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], oinv, ot, rows, positions=pos, q_start=500, k_start=0)
     assert_bf16(errors(*gather_gpu(o, lse, rows), Or, Lr))
 
 
@@ -193,7 +226,7 @@ def test_fully_masked_rows_and_empty_inputs(dtype):
 
 def test_rotate_k_in_kernel_unsupported_on_tensor_core_path():
     q, k, v = make_qkv(1, 16, 2, 1, 128, torch.bfloat16, seed=11, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    inv, t, oinv, ot = schedule(_lib.PLAIN, 1e4, 128, 10, 10)
     with pytest.raises(_lib.RcxError) as e:
         _lib.attn_blockwise_fwd(q, k, v, inv_freq=inv, rope_flags=_lib.ROTATE_K)
     assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
@@ -230,6 +263,34 @@ def test_merge_partials(out):
     assert np.abs(np64(gl)[fin] - rl[fin]).max() <= 1e-5
 
 
+@pytest.mark.parametrize("dtype,d,out_bf16", [(torch.bfloat16, 128, True), (torch.bfloat16, 128, False),
+                                              (torch.float32, 64, False)])
+def test_attention_merged_into_previous_partial(dtype, d, out_bf16):
+    # Three key blocks visited in ring order 2, 1, 0 for query rows of block 2:
+    # the first call writes the fp32 accumulator, the second merges in place
+    # in the epilogue, the third merges into the final output.
+    N, nb = 600, 200
+    q, k, v = make_qkv(1, N, 4, 2, d, dtype, seed=33, device=DEV)
+    inv, t, oinv, ot = schedule(_lib.YARN, 1e4, d, 256, 2048)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)
+    qs = q[:, 2 * nb:].contiguous()
+    acc = torch.empty(1, nb, 4, d, dtype=torch.float32, device=DEV)
+    lacc = torch.empty(1, 4, nb, dtype=torch.float32, device=DEV)
+    out = torch.empty(1, nb, 4, d, dtype=torch.bfloat16 if out_bf16 else torch.float32, device=DEV)
+    lse = torch.empty(1, 4, nb, dtype=torch.float32, device=DEV)
+    kw = dict(window=300, n_sink=3, temperature=t, q_start=2 * nb, inv_freq=inv, rope_flags=_lib.ROTATE_Q)
+    blk = lambda x, b: x[:, b * nb:(b + 1) * nb].contiguous()
+    _lib.attn_blockwise_fwd(qs, blk(krot, 2), blk(v, 2), acc, lacc, k_start=2 * nb, **kw)
+    _lib.attn_blockwise_merge_fwd(qs, blk(krot, 1), blk(v, 1), acc, lacc, acc, lacc, k_start=nb, **kw)
+    _lib.attn_blockwise_merge_fwd(qs, blk(krot, 0), blk(v, 0), out, lse, acc, lacc, k_start=0, **kw)
+    torch.cuda.synchronize()
+    rows = all_rows(nb, 4)
+    Or, Lr = oracle_rows(qs[0], k[0], v[0], oinv, ot, rows, 300, 3, q_start=2 * nb, k_start=0)
+    err = errors(*gather_gpu(out, lse, rows), Or, Lr)
+    (assert_bf16 if (dtype == torch.bfloat16 or out_bf16) else assert_f32)(err)
+
+
 # ----------------------------------------------------------------------- ring
 
 @pytest.mark.parametrize("dtype,d,N,kv_block,window,n_sink", [
@@ -237,12 +298,12 @@ def test_merge_partials(out):
     (torch.float32, 64, 512, 64, 0, 0), (torch.float32, 64, 300, 128, 50, 2)])
 def test_ring_driver_matches_oracle(dtype, d, N, kv_block, window, n_sink):
     q, k, v = make_qkv(1, N, 4, 2, d, dtype, seed=13, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.NTK, 1e4, d, 256, 1024)
+    inv, t, oinv, ot = schedule(_lib.NTK, 1e4, d, 256, 1024)
     o, lse = _lib.ring_attn_fwd(q, k, v, kv_block=kv_block, window=window, n_sink=n_sink, temperature=t,
                                 inv_freq=inv, rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
     torch.cuda.synchronize()
     rows = all_rows(N, 4)
-    Or, Lr = oracle_rows(q[0], k[0], v[0], inv, t, rows, window, n_sink)
+    Or, Lr = oracle_rows(q[0], k[0], v[0], oinv, ot, rows, window, n_sink)
     err = errors(*gather_gpu(o, lse, rows), Or, Lr)
     (assert_bf16 if dtype == torch.bfloat16 else assert_f32)(err)
 
@@ -250,7 +311,7 @@ def test_ring_driver_matches_oracle(dtype, d, N, kv_block, window, n_sink):
 def test_ring_equals_single_call_bf16():
     N = 1024
     q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=14, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 256, 2048)
+    inv, t, oinv, ot = schedule(_lib.NTK, 5e5, 128, 256, 2048)
     o1, l1 = _lib.ring_attn_fwd(q, k, v, kv_block=256, temperature=t, inv_freq=inv,
                                 rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
     krot = torch.empty_like(k)
@@ -265,7 +326,7 @@ def test_ring_equals_single_call_bf16():
 def test_ring_host_buffers_entry_point():
     N = 512
     q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=15, device="cpu")
-    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 256, 1024)
+    inv, t, oinv, ot = schedule(_lib.NTK, 5e5, 128, 256, 1024)
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
     oh = torch.empty_like(qh).pin_memory()
     lh = torch.empty(1, 4, N, dtype=torch.float32).pin_memory()
@@ -296,6 +357,30 @@ def test_bounded_wait_timeout_reports_and_context_survives():
     assert torch.isfinite(o.float()).all()
 
 
+def test_host_entry_point_reports_device_timeout():
+    # The synchronous host-buffer entry point reads the device status words
+    # itself: a bounded wait that ran out returns RCX_ERR_DEVICE_TIMEOUT from
+    # the call, and the word is cleared for the next call.
+    N = 256
+    q, k, v = make_qkv(1, N, 2, 1, 128, torch.bfloat16, seed=16, device="cpu")
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    inv, t, _, _ = schedule(_lib.NTK, 5e5, 128, 256, 1024)
+    assert _lib.device_status() == 0
+    _lib.debug_inject_wait_timeout(20000)
+    try:
+        with pytest.raises(_lib.RcxError) as e:
+            _lib.ring_attn_fwd_host(qh, kh, vh, oh, None, kv_block=128, temperature=t, inv_freq=inv,
+                                    rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+        assert e.value.status == _lib.RCX_ERR_DEVICE_TIMEOUT
+    finally:
+        _lib.debug_inject_wait_timeout(0)
+    assert _lib.device_status() == 0
+    _lib.ring_attn_fwd_host(qh, kh, vh, oh, None, kv_block=128, temperature=t, inv_freq=inv,
+                            rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    assert torch.isfinite(oh.float()).all()
+
+
 # --------------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("B,Nk,Hq,Hkv,window,n_sink,qoff", [
@@ -304,7 +389,7 @@ def test_bounded_wait_timeout_reports_and_context_survives():
 def test_decode_split_kv_matches_oracle(B, Nk, Hq, Hkv, window, n_sink, qoff):
     qf, _, _ = make_qkv(B, 1, Hq, Hkv, 128, torch.bfloat16, seed=20, device=DEV)
     _, k, v = make_qkv(B, Nk, Hq, Hkv, 128, torch.bfloat16, seed=21, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 8192, 131072)
+    inv, t, oinv, ot = schedule(_lib.NTK, 5e5, 128, 8192, 131072)
     krot = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, k_out=krot)                 # the cache holds rotated keys
     q_index = Nk - 1 + qoff                                    # newest token (or later: all keys visible)
@@ -316,7 +401,7 @@ def test_decode_split_kv_matches_oracle(B, Nk, Hq, Hkv, window, n_sink, qoff):
     torch.cuda.synchronize()
     for b in range(B):
         rows = {h: np.array([0]) for h in range(Hq)}
-        Or, Lr = oracle_rows(qf[b], k[b], v[b], inv, t, rows, window, n_sink, q_start=q_index, k_start=0)
+        Or, Lr = oracle_rows(qf[b], k[b], v[b], oinv, ot, rows, window, n_sink, q_start=q_index, k_start=0)
         Og = {h: np64(o[b, 0, h, :])[None] for h in range(Hq)}
         Lg = {h: np.array([float(lse[b, h, 0])]) for h in range(Hq)}
         err = errors(Og, Lg, Or, Lr)
@@ -329,7 +414,7 @@ def test_decode_8_byte_rows_matches_oracle(Hq, Hkv, window, n_sink):
     Nk = 2500
     qf, _, _ = make_qkv(1, 1, Hq, Hkv, 128, torch.bfloat16, seed=25, device=DEV)
     _, k, v = make_qkv(1, Nk, Hq, Hkv, 128, torch.bfloat16, seed=26, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.YARN, 1e4, 128, 4096, 32768)
+    inv, t, oinv, ot = schedule(_lib.YARN, 1e4, 128, 4096, 32768)
     krot = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, k_out=krot)
     kp = torch.zeros(1, Nk, Hkv, 132, dtype=torch.bfloat16, device=DEV)
@@ -343,7 +428,7 @@ def test_decode_8_byte_rows_matches_oracle(Hq, Hkv, window, n_sink):
                                     inv_freq=inv, rope_flags=_lib.ROTATE_Q)
     torch.cuda.synchronize()
     rows = {h: np.array([0]) for h in range(Hq)}
-    Or, Lr = oracle_rows(qf[0], k[0], v[0], inv, t, rows, window, n_sink, q_start=Nk - 1, k_start=0)
+    Or, Lr = oracle_rows(qf[0], k[0], v[0], oinv, ot, rows, window, n_sink, q_start=Nk - 1, k_start=0)
     for oo, ll in ((o, lse), (o2, lse2)):
         Og = {h: np64(oo[0, 0, h, :])[None] for h in range(Hq)}
         Lg = {h: np.array([float(ll[0, h, 0])]) for h in range(Hq)}
@@ -358,7 +443,7 @@ def test_decode_rejects_rotate_k_and_bad_group():
         _lib.attn_decode_fwd(q, kc, vc)
     assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
     q2, _, _ = make_qkv(1, 1, 4, 2, 128, torch.bfloat16, seed=24, device=DEV)
-    inv, _ = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    inv, _, oinv, _ = schedule(_lib.PLAIN, 1e4, 128, 10, 10)
     with pytest.raises(_lib.RcxError) as e:
         _lib.attn_decode_fwd(q2, kc, vc, inv_freq=inv, rope_flags=_lib.ROTATE_K)
     assert e.value.status == _lib.RCX_ERR_UNSUPPORTED
@@ -366,11 +451,11 @@ def test_decode_rejects_rotate_k_and_bad_group():
 
 # ------------------------------------------------------------ batch > 1, G = 8
 
-def _oracle_batch(q, k, v, inv, t, window=0, n_sink=0):
+def _oracle_batch(q, k, v, oinv, ot, window=0, n_sink=0):
     out = []
     for b in range(q.shape[0]):
         rows = all_rows(q.shape[1], q.shape[2])
-        out.append((rows, *oracle_rows(q[b], k[b], v[b], inv, t, rows, window, n_sink)))
+        out.append((rows, *oracle_rows(q[b], k[b], v[b], oinv, ot, rows, window, n_sink)))
     return out
 
 
@@ -378,13 +463,13 @@ def _oracle_batch(q, k, v, inv, t, window=0, n_sink=0):
 def test_bf16_tensor_core_batch2(Hq, Hkv, window, n_sink):
     B, N = 2, 700
     q, k, v = make_qkv(B, N, Hq, Hkv, 128, torch.bfloat16, seed=30, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.YARN, 1e4, 128, 512, 4096)
+    inv, t, oinv, ot = schedule(_lib.YARN, 1e4, 128, 512, 4096)
     krot = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, k_out=krot)
     o, lse = _lib.attn_blockwise_fwd(q, krot, v, temperature=t, inv_freq=inv, rope_flags=_lib.ROTATE_Q,
                                      window=window, n_sink=n_sink)
     torch.cuda.synchronize()
-    for b, (rows, Or, Lr) in enumerate(_oracle_batch(q, k, v, inv, t, window, n_sink)):
+    for b, (rows, Or, Lr) in enumerate(_oracle_batch(q, k, v, oinv, ot, window, n_sink)):
         Og = {h: np64(o[b, r, h, :]) for h, r in rows.items()}
         Lg = {h: lse[b, h, r].cpu().numpy().astype(np.float64) for h, r in rows.items()}
         assert_bf16(errors(Og, Lg, Or, Lr))
@@ -394,11 +479,11 @@ def test_bf16_tensor_core_batch2(Hq, Hkv, window, n_sink):
 def test_ring_batch2(dtype, d):
     B, N = 2, 640
     q, k, v = make_qkv(B, N, 8, 2, d, dtype, seed=31, device=DEV)
-    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, d, 256, 2048)
+    inv, t, oinv, ot = schedule(_lib.NTK, 5e5, d, 256, 2048)
     o, lse = _lib.ring_attn_fwd(q, k, v, kv_block=256, temperature=t, inv_freq=inv,
                                 rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
     torch.cuda.synchronize()
-    for b, (rows, Or, Lr) in enumerate(_oracle_batch(q, k, v, inv, t)):
+    for b, (rows, Or, Lr) in enumerate(_oracle_batch(q, k, v, oinv, ot)):
         Og = {h: np64(o[b, r, h, :]) for h, r in rows.items()}
         Lg = {h: lse[b, h, r].cpu().numpy().astype(np.float64) for h, r in rows.items()}
         (assert_bf16 if dtype == torch.bfloat16 else assert_f32)(errors(Og, Lg, Or, Lr))
@@ -408,10 +493,10 @@ def test_rope_apply_batch_wrap_in_chunk():
     # N smaller than a bulk chunk: chunks straddle batch entries (direct angles).
     B, N = 5, 3
     q, k, _ = make_qkv(B, N, 2, 8, 128, torch.bfloat16, seed=32, device=DEV)
-    inv, _ = _lib.rope_freqs(_lib.PLAIN, 1e4, 128, 10, 10)
+    inv, _, oinv, _ = schedule(_lib.PLAIN, 1e4, 128, 10, 10)
     ko = torch.empty_like(k)
     _lib.rope_apply(None, k, inv, k_out=ko)
     torch.cuda.synchronize()
     for b in range(B):
-        ref = orc.rope_rotate(np64(k[b]), np.arange(N), inv)
+        ref = orc.rope_rotate(np64(k[b]), np.arange(N), oinv)
         assert np.all(np.abs(np64(ko[b]) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)

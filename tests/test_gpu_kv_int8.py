@@ -11,7 +11,7 @@ import torch
 from oracle import rcx_oracle as orc
 from rope_context_extension_scaled_b200 import _lib
 from rope_context_extension_scaled_b200.inputs import make_qkv
-from tests._parity import errors, np64
+from tests._parity import schedule, errors, np64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -93,7 +93,7 @@ def test_decode_int8_matches_oracle(B, Nk, Hq, Hkv, window, n_sink, qoff):
     qf, _, _ = make_qkv(B, 1, Hq, Hkv, 128, torch.bfloat16, seed=70, device=DEV)
     k = _k_cache(B, Nk, Hkv, seed=71)
     v = _v_cache(B, Nk, Hkv, seed=72)
-    inv, t = _lib.rope_freqs(_lib.YARN, 5e5, 128, 8192, 131072)
+    inv, t, oinv, ot = schedule(_lib.YARN, 5e5, 128, 8192, 131072)
     kc, ks = _lib.kv_quantize_int8(k)
     vc, vs = _lib.kv_quantize_int8(v)
     q_index = Nk - 1 + qoff
@@ -101,7 +101,7 @@ def test_decode_int8_matches_oracle(B, Nk, Hq, Hkv, window, n_sink, qoff):
                                        q_index=q_index, inv_freq=inv, rope_flags=_lib.ROTATE_Q)
     torch.cuda.synchronize()
     for b in range(B):
-        Or, Lr = _oracle_decode(qf[b], k[b], v[b], inv, t, q_index, window, n_sink)
+        Or, Lr = _oracle_decode(qf[b], k[b], v[b], oinv, ot, q_index, window, n_sink)
         Og = {h: np64(o[b, 0, h, :])[None] for h in range(Hq)}
         Lg = {h: np.array([float(lse[b, h, 0])]) for h in range(Hq)}
         Ors = {h: Or[h][None] for h in range(Hq)}
@@ -131,14 +131,14 @@ def test_decode_int8_full_size_cache():
     qf, _, _ = make_qkv(1, 1, 64, 8, 128, torch.bfloat16, seed=90, device=DEV)
     k = _k_cache(1, Nk, 8, seed=91)
     v = _v_cache(1, Nk, 8, seed=92)
-    inv, t = _lib.rope_freqs(_lib.NTK, 5e5, 128, 8192, Nk)
+    inv, t, oinv, ot = schedule(_lib.NTK, 5e5, 128, 8192, Nk)
     kc, ks = _lib.kv_quantize_int8(k)
     vc, vs = _lib.kv_quantize_int8(v)
     o, lse = _lib.attn_decode_int8_fwd(qf, kc, ks, vc, vs, temperature=t, inv_freq=inv, rope_flags=_lib.ROTATE_Q)
     torch.cuda.synchronize()
     for g in (0, 7):                                       # KV groups 0 and 7 (query heads 0-7, 56-63)
         hs = slice(8 * g, 8 * g + 8)
-        Or, Lr = _oracle_decode(qf[0][:, hs], k[0][:, g:g + 1], v[0][:, g:g + 1], inv, t, Nk - 1, 0, 0)
+        Or, Lr = _oracle_decode(qf[0][:, hs], k[0][:, g:g + 1], v[0][:, g:g + 1], oinv, ot, Nk - 1, 0, 0)
         Og = {h: np64(o[0, 0, 8 * g + h, :])[None] for h in range(8)}
         Lg = {h: np.array([float(lse[0, 8 * g + h, 0])]) for h in range(8)}
         err = errors(Og, Lg, {h: Or[h][None] for h in range(8)}, {h: np.array([Lr[h]]) for h in range(8)})
