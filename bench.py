@@ -4,8 +4,8 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input
 (K rotation, tensor-core attention with the Q rotation fused in its tile load,
-and for ring workloads the ring schedule with its LSE merges), through the C
-ABI.  The default workload is the 1M-token ring configuration (64 Q / 8 KV
+and for ring workloads the ring schedule, whose LSE merges run in the epilogue
+of each later block's attention), through the C ABI.  The default workload is the 1M-token ring configuration (64 Q / 8 KV
 heads, d 128, NTK s = 128, 16 ring blocks of 65,536 keys); the 128K sliding-
 window configuration is timed in the same run and reported under "secondary".
 
@@ -399,6 +399,15 @@ def run_ours(args, w):
                                 "pct_hbm": 100.0 * kv8_bytes / (d8_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                 "tokens_per_s": world * w.B / (d8_ms * 1e-3),
                                 "bytes_per_step": kv8_bytes}
+        # the append path: quantising the bf16 K cache (read bf16, write codes and scales)
+        kq_out = torch.empty_like(kc)
+        ksc_out = torch.empty_like(ks)
+        q_ms = time_steps(lambda: _lib.kv_quantize_int8(k, codes=kq_out, scale=ksc_out), 10, 3, stream, dist, world)
+        q_bytes = k.numel() * k.element_size() + kq_out.numel() + 4 * ksc_out.numel()
+        decode["int8_quantize"] = {"workload": f"quantise the {w.N}-token K cache ({w.Hkv} heads)", "ms": q_ms,
+                                   "gbs": q_bytes / (q_ms * 1e-3) / 1e9,
+                                   "pct_hbm": 100.0 * q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del kq_out, ksc_out
         del qd, od, ld, wsd, kc, ks, vc, vs, ws8
     peak_key = "bf16_tflops_sustained" if ms > 1000 else "bf16_tflops"
     peak = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])

@@ -1,6 +1,7 @@
 // Host side of the tensor-core attention kernel (attn_tc.cuh): TMA tensor
 // maps, launch configuration, the bounded-wait test hook and the status word.
 #include <cuda.h>
+#include <algorithm>
 #include <cstring>
 #include "launch.h"
 #include "attn_tc.cuh"
@@ -77,6 +78,14 @@ int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tensor& k, 
   const int64_t items = (int64_t)p.n_rb * p.n_hg * a.q.B;
   if (items <= 0) return RCX_OK;
   if (items > 0x7fffffff) return RCX_ERR_UNSUPPORTED;
+  // the kernel's tile walk and row arithmetic are 32-bit: global token
+  // indices (and the window, sink and block sizes) stay below 2^31
+  const int64_t lim = 0x7fffffffll - 2 * kTcBM;
+  if (a.q_start + a.q.N > lim || a.k_start + a.k.N > lim || a.kv_block > lim || a.window > lim || a.n_sink > lim)
+    return RCX_ERR_UNSUPPORTED;
+  p.n_items = (int)items;
+  // persistent: at most one CTA per SM, each walking items blockIdx.x + k * gridDim.x
+  const int grid = (int)std::min<int64_t>(items, (int64_t)sm_count());
   const cudaError_t ea = o.dtype == RCX_BF16
                              ? cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmTotal)
@@ -85,9 +94,9 @@ int attn_tc_launch(const AttnArgs& a, const rcx_tensor& q, const rcx_tensor& k, 
   if (ea != cudaSuccess) return RCX_ERR_CUDA;
   LaunchScope scope(RCX_KERNEL_ATTN_TC, stream);
   if (o.dtype == RCX_BF16)
-    attn_tc_kernel<__nv_bfloat16><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
+    attn_tc_kernel<__nv_bfloat16><<<grid, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
   else
-    attn_tc_kernel<float><<<(unsigned)items, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
+    attn_tc_kernel<float><<<grid, kTcThreads, kSmTotal, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RCX_OK : RCX_ERR_CUDA;
 }

@@ -47,9 +47,12 @@ int decode_combine_launch(const DecodeArgs& a, int out_dtype, int grid, cudaStre
   return launch_status();
 }
 
-int quantize_i8_launch(const QuantArgs& a, int grid, cudaStream_t stream) {
+int quantize_i8_launch(const QuantArgs& a, bool rows16, int grid, cudaStream_t stream) {
   LaunchScope scope(RCX_KERNEL_DECODE, stream);
-  kv_quantize_int8_kernel<<<grid, 256, 0, stream>>>(a);
+  if (rows16)
+    kv_quantize_int8_h16_kernel<<<grid, 256, 0, stream>>>(a);
+  else
+    kv_quantize_int8_kernel<<<grid, 256, 0, stream>>>(a);
   return launch_status();
 }
 

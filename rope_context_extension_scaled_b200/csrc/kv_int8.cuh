@@ -14,8 +14,13 @@
 //    becomes an exact fp16 in three integer/half instructions: the byte with
 //    its sign bit flipped (u = code + 128) is placed under the exponent
 //    pattern of 1024, which reads as 1024 + u, and 1152 is subtracted;
-//  * K codes go into S^T = Kq Q^T unscaled; each key's scale then multiplies
-//    its row of S^T in fp32;
+//  * K codes go into S^T = Kq Q^T unscaled and without the subtraction, i.e.
+//    as code + 1152 (two instructions per pair of codes): the product then
+//    carries 1152 sum_d q_d per query head, which is removed from S^T in fp32
+//    (the products are exact in fp32 and |S'| stays near 1e4, so the
+//    cancellation costs about 1e-5 of the logit); each key's scale then
+//    multiplies its row of S^T.  The V path keeps the subtraction: there the
+//    offset would grow with the number of keys summed into O;
 //  * V codes go into O^T += Vq^T P'^T unscaled, with each key's V scale folded
 //    into P: P' = p * s_v / s_max, where s_max is the largest V scale the warp
 //    has met so far (so P' stays in [0, 1], clear of fp16 subnormals).  When
@@ -96,6 +101,78 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const Quan
   }
 }
 
+// Half-warp per row, for rows whose bf16 values and codes are 16- and 8-byte
+// aligned: lane l of a half holds dims 8l .. 8l + 7 (one 16-byte load, so a
+// row is one coalesced 256-byte read), the row max takes four shuffles within
+// the half, and each lane stores its 8 codes as one 8-byte word.  A warp has
+// kQRowsH row pairs in flight per pass, all loads issued before any
+// arithmetic.  Same IEEE fp32 decisions as kv_quantize_int8_kernel, so the
+// codes and scales are identical.
+constexpr int kQRowsH = 4;
+
+__device__ __forceinline__ void quant_row_offsets(const QuantArgs& a, int64_t r, int64_t& off_x, int64_t& off_c) {
+  int64_t h, n, b;
+  if (a.rows < (int64_t(1) << 31)) {          // 32-bit index arithmetic (the usual case)
+    const uint32_t r32 = (uint32_t)r, H32 = (uint32_t)a.x.H, N32 = (uint32_t)a.x.N;
+    const uint32_t t32 = r32 / H32;
+    h = r32 - t32 * H32;
+    n = t32 % N32;
+    b = t32 / N32;
+  } else {
+    h = r % a.x.H;
+    n = (r / a.x.H) % a.x.N;
+    b = r / (a.x.H * a.x.N);
+  }
+  off_x = b * a.x.sb + n * a.x.sn + h * a.x.sh;
+  off_c = b * a.c.sb + n * a.c.sn + h * a.c.sh;
+}
+
+static __global__ void __launch_bounds__(256) kv_quantize_int8_h16_kernel(const QuantArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4, hl = lane & 15;
+  const int64_t pairs = (a.rows + 1) / 2;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
+  const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  for (int64_t p0 = w0; p0 < pairs; p0 += kQRowsH * nwarps) {
+    uint4 u[kQRowsH];
+    int64_t off_c[kQRowsH];
+#pragma unroll
+    for (int i = 0; i < kQRowsH; ++i) {
+      const int64_t p = p0 + i * nwarps;
+      int64_t r = 2 * (p < pairs ? p : p0) + half;
+      if (r >= a.rows) r = a.rows - 1;               // odd row count: the last half repeats a row, stores nothing
+      int64_t off_x;
+      quant_row_offsets(a, r, off_x, off_c[i]);
+      u[i] = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.x.ptr) + off_x + 8 * hl);
+    }
+#pragma unroll
+    for (int i = 0; i < kQRowsH; ++i) {
+      const int64_t p = p0 + i * nwarps;
+      if (p >= pairs) break;                         // warp-uniform
+      const int64_t r = 2 * p + half;
+      const float2 x01 = bf2_to_f2(u[i].x), x23 = bf2_to_f2(u[i].y), x45 = bf2_to_f2(u[i].z), x67 = bf2_to_f2(u[i].w);
+      const float v[8] = {x01.x, x01.y, x23.x, x23.y, x45.x, x45.y, x67.x, x67.y};
+      float am = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+      const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        int q = __float2int_rn(__fmul_rn(v[e], inv));
+        q = q > 127 ? 127 : (q < -127 ? -127 : q);
+        w[e >> 2] |= (uint32_t)(q & 0xff) << (8 * (e & 3));
+      }
+      if (r < a.rows) {
+        *reinterpret_cast<uint2*>(reinterpret_cast<int8_t*>(a.c.ptr) + off_c[i] + 8 * hl) = make_uint2(w[0], w[1]);
+        if (hl == 0) a.scale[r] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- decode
 
 constexpr int kDqWarps = 8;
@@ -118,6 +195,13 @@ __device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint3
 __device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Two int8 codes (bytes 0 and 2 of u ^ 0x80808080 selected by sel) -> the
+// exact fp16 pair code + 1152 (the byte u = code + 128 under the exponent
+// pattern of 1024); the K path keeps the offset and removes it from S.
+__device__ __forceinline__ uint32_t codes_to_h2_off(uint32_t u_flipped, uint32_t sel) {
+  return __byte_perm(u_flipped, 0x64646464u, sel);                  // halves 0x64uu = 1024 + u
 }
 
 // Two int8 codes (bytes 0 and 2 of u ^ 0x80808080 selected by sel) -> exact fp16 pair.
@@ -161,6 +245,25 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
   } else {
 #pragma unroll
     for (int kc = 0; kc < 8; ++kc) qb[kc][0] = qb[kc][1] = 0u;
+  }
+
+  // K codes enter the S^T product as code + 1152, so S'^T = S^T + 1152 sum_d q_d
+  // per query head; qs[h] (h = 0, 1: heads 2c, 2c + 1, this lane's columns)
+  // is that sum over the same fp16 q values the MMA reads.
+  float qs[2];
+  {
+    float part = 0.f;
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&qb[kc][hf]);
+        part += __low2float(h) + __high2float(h);
+      }
+    part += __shfl_xor_sync(0xffffffffu, part, 1);     // lanes 4g .. 4g + 3 hold head g
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    qs[0] = __shfl_sync(0xffffffffu, part, 8 * c) * 1152.f;
+    qs[1] = __shfl_sync(0xffffffffu, part, 8 * c + 4) * 1152.f;
   }
 
   // ---- this warp's key range, in 16-key tiles from k_lo
@@ -253,8 +356,8 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
 #pragma unroll
     for (int kc = 0; kc < 8; ++kc) {
       const uint32_t fa = kw[0][kc] ^ 0x80808080u, fb = kw[1][kc] ^ 0x80808080u;
-      const uint32_t af[4] = {codes_to_h2(fa, 0x4140), codes_to_h2(fb, 0x4140), codes_to_h2(fa, 0x4342),
-                              codes_to_h2(fb, 0x4342)};
+      const uint32_t af[4] = {codes_to_h2_off(fa, 0x4140), codes_to_h2_off(fb, 0x4140), codes_to_h2_off(fa, 0x4342),
+                              codes_to_h2_off(fb, 0x4342)};
       mma_f16_16816(sacc, af, qb[kc][0], qb[kc][1]);
     }
     // key scales, online softmax per head over keys t0 + g, t0 + g + 8
@@ -272,10 +375,10 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
     const bool va = ja < k_hi && mask_visible(qi, ja, a.window, a.n_sink);
     const bool vb = jb < k_hi && mask_visible(qi, jb, a.window, a.n_sink);
     float sv[4];
-    sv[0] = va ? sacc[0] * ska * a.scale_log2 : -INFINITY;
-    sv[1] = va ? sacc[1] * ska * a.scale_log2 : -INFINITY;
-    sv[2] = vb ? sacc[2] * skb * a.scale_log2 : -INFINITY;
-    sv[3] = vb ? sacc[3] * skb * a.scale_log2 : -INFINITY;
+    sv[0] = va ? (sacc[0] - qs[0]) * ska * a.scale_log2 : -INFINITY;
+    sv[1] = va ? (sacc[1] - qs[1]) * ska * a.scale_log2 : -INFINITY;
+    sv[2] = vb ? (sacc[2] - qs[0]) * skb * a.scale_log2 : -INFINITY;
+    sv[3] = vb ? (sacc[3] - qs[1]) * skb * a.scale_log2 : -INFINITY;
     float p[4], beta[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {

@@ -245,7 +245,7 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
         b.d_chunks = (int)(D * elem_size(dtype) / 16);
         for (int j = 0; j < b.pairs; ++j) b.f.theta[j] = inv_freq[j];
         const int64_t chunks = (b.n_tok + b.tok_per_chunk - 1) / b.tok_per_chunk;
-        const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 2);
+        const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 4);
         const int st = rope_bulk_launch(b, dtype, grid, smem, stream);
         if (st) return st;
       }
@@ -518,8 +518,11 @@ int quantize_i8_impl(const rcx_tensor& x, const rcx_tensor& c, float* scale, cud
   a.c = make_view(c);
   a.scale = scale;
   a.rows = rows;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + 7) / 8, (int64_t)sm_count() * 8));
-  return quantize_i8_launch(a, grid, stream);
+  const bool rows16 = aligned_rows(x, 16) && aligned_rows(c, 8);
+  const int64_t per_cta = rows16 ? 16 : 8;      // rows a CTA covers per pass (two or one per warp)
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + per_cta - 1) / per_cta,
+                                                              (int64_t)sm_count() * 8));
+  return quantize_i8_launch(a, rows16, grid, stream);
 }
 
 int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scale, const rcx_tensor& v,

@@ -172,20 +172,22 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_apply_kernel(const RopeA
 // one is rotated and stored, so every thread keeps 2 x kRopePieces 16-byte
 // loads in flight; one barrier per chunk publishes the chunk's angles.
 //
-// Angles with consecutive positions (positions == NULL; position = token
-// index within its batch entry): cos/sin of (n0 + t) theta come from the
-// angle-addition identity applied once to two exact values, the chunk's base
-// angle n0 theta (one precise angle per pair per chunk) and the step angle
-// t theta (t < T, a table built once per CTA).  Both come from rope_cos_sin,
-// so the applied angle is within a few 1e-7 rad of m theta and there is no
-// recurrence whose rounding grows with t.  With explicit positions every
-// (token, pair) angle of the chunk is computed directly into a table; a chunk
-// that crosses into the next batch entry computes its angles per piece.
+// Each chunk's (token, pair) cos/sin table is built while the previous chunk
+// is rotated (double buffer), so rotating a piece costs table loads and four
+// rotations.  With consecutive positions (positions == NULL; position = token
+// index within its batch entry) the entry for token t of a chunk starting at
+// n0 comes from the angle-addition identity applied once to two exact values,
+// the base angle n0 theta (computed by each thread for the pair it owns) and
+// the step angle t theta (t < T, a table built once per CTA).  Both come from
+// rope_cos_sin, so the applied angle is within a few 1e-7 rad of m theta and
+// there is no recurrence whose rounding grows with t.  With explicit
+// positions, or in a chunk that crosses into the next batch entry, every
+// entry is computed directly.
 
-constexpr int kRopePieces = 8;                         // 16-byte pieces per thread per chunk
-constexpr int kRopeBulkBytes = kRopeThreads * kRopePieces * 16;   // 32 KB chunk
+constexpr int kRopePieces = 4;                         // 16-byte pieces per thread per chunk
+constexpr int kRopeBulkBytes = kRopeThreads * kRopePieces * 16;   // 16 KB chunk
 constexpr int kRopeBulkTab = kRopeMaxAngles / 2;       // float2 entries of one angle table (>= T * pairs)
-constexpr size_t kRopeBulkSmem = 3 * kRopeBulkTab * sizeof(float2);
+constexpr size_t kRopeBulkSmem = 3 * kRopeBulkTab * sizeof(float2);   // step table + two chunk tables
 
 struct RopeBulkArgs {
   const void* in;
@@ -208,18 +210,17 @@ __device__ __forceinline__ float2 cs_add(float2 a, float2 b) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBulkArgs a) {
+__global__ void __launch_bounds__(kRopeThreads, 4) rope_bulk_kernel(const RopeBulkArgs a) {
   constexpr int kElems = 16 / sizeof(T);
   constexpr int kPairsPerChunk = kElems / 2;
   extern __shared__ __align__(16) float2 rb_tabs[];     // [3][kRopeBulkTab]
   const int tid = threadIdx.x;
   const int pairs = a.pairs;
   const bool dense_pos = a.positions == nullptr;
-  // dense positions: tabs[0] = step table [T][pairs], tabs[1] = base angles [2][pairs];
-  // explicit positions: tabs[1], tabs[2] = direct tables [T][pairs] (double buffer)
+  // tabs[0] = step table [T][pairs] (consecutive positions); tabs[1 + buf] =
+  // (cos, sin) of the chunk's entries [t][pairs], double-buffered
   float2* step_tab = rb_tabs;
-  float2* base_tab = rb_tabs + kRopeBulkTab;
-  auto direct_tab = [&](int buf) { return rb_tabs + (1 + buf) * kRopeBulkTab; };
+  auto chunk_tab = [&](int buf) { return rb_tabs + (1 + buf) * kRopeBulkTab; };
 
   const int64_t n_chunks = (a.n_tok + a.tok_per_chunk - 1) / a.tok_per_chunk;
   const int64_t step = gridDim.x;
@@ -227,47 +228,50 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBu
     const int64_t left = a.n_tok - c * a.tok_per_chunk;
     return (int)(left < a.tok_per_chunk ? left : a.tok_per_chunk);
   };
-  // First token n0 (within its batch entry) of chunk c; true when the chunk
-  // stays in one batch entry.
-  auto in_one_entry = [&](int64_t c, int64_t& n0) {
-    const int64_t t0 = c * a.tok_per_chunk;
-    n0 = t0 - (t0 / a.N) * a.N;
-    return n0 + chunk_tokens(c) <= a.N;
-  };
-  // Angles chunk c needs, into buffer `buf`.  Threads 0, 4, 8, ... take the
-  // base angles, so the extra sincos work spreads over all warps.
+  // Table of chunk c into buffer `buf`, entry e = t * pairs + p.  When 256 is
+  // a multiple of pairs, a thread's entries share one pair p, so each thread
+  // computes the base angle of its own pair (the redundant sincos keeps every
+  // thread's share of the work equal ahead of the next barrier).
+  const bool fixed_pair = (kRopeThreads % pairs) == 0;
   auto prepare = [&](int64_t c, int buf) {
-    int64_t n0;
-    const bool one = in_one_entry(c, n0);
-    if (dense_pos) {
-      if (one)
-        for (int j = tid; j < 4 * pairs; j += kRopeThreads)
-          if ((j & 3) == 0) {
-            float cc, sn;
-            rope_cos_sin(n0, a.f.theta[j >> 2], cc, sn);
-            base_tab[buf * kMaxPairs + (j >> 2)] = make_float2(cc, sn);
-          }
+    const int ntok = chunk_tokens(c);
+    const int64_t t0 = c * a.tok_per_chunk;
+    const int64_t n0 = t0 - (t0 / a.N) * a.N;
+    const bool consecutive = dense_pos && n0 + ntok <= a.N;
+    float2* tab = chunk_tab(buf);
+    const int total = ntok * pairs;
+    if (consecutive && fixed_pair) {
+      if (tid < total) {
+        float bc, bs;
+        rope_cos_sin(n0, a.f.theta[tid % pairs], bc, bs);
+        const float2 base = make_float2(bc, bs);
+        for (int e = tid; e < total; e += kRopeThreads) tab[e] = cs_add(base, step_tab[e]);
+      }
       return;
     }
-    const int ntok = chunk_tokens(c);
-    float2* tab = direct_tab(buf);
-    for (int e = tid; e < ntok * pairs; e += kRopeThreads) {
+    for (int e = tid; e < total; e += kRopeThreads) {
       const int t = e / pairs, p = e - t * pairs;
-      int64_t n = n0 + t;
-      while (n >= a.N) n -= a.N;
       float cc, sn;
-      rope_cos_sin(a.positions[n], a.f.theta[p], cc, sn);
-      tab[t * pairs + p] = make_float2(cc, sn);
+      if (consecutive) {
+        rope_cos_sin(n0, a.f.theta[p], cc, sn);
+        tab[e] = cs_add(make_float2(cc, sn), step_tab[e]);
+      } else {
+        int64_t n = n0 + t;
+        while (n >= a.N) n -= a.N;
+        rope_cos_sin(a.positions ? a.positions[n] : n, a.f.theta[p], cc, sn);
+        tab[e] = make_float2(cc, sn);
+      }
     }
   };
 
-  // This thread's pieces: token and first pair of piece e = tid + 256 k.
-  int pt[kRopePieces], pp[kRopePieces];
+  // This thread's pieces: table offset (token * pairs + first pair) of piece
+  // e = tid + 256 k.
+  int pofs[kRopePieces];
 #pragma unroll
   for (int k = 0; k < kRopePieces; ++k) {
     const int e = tid + k * kRopeThreads;
-    pt[k] = e / a.row_chunks;
-    pp[k] = ((e - pt[k] * a.row_chunks) % a.d_chunks) * kPairsPerChunk;
+    const int t = e / a.row_chunks;
+    pofs[k] = t * pairs + ((e - t * a.row_chunks) % a.d_chunks) * kPairsPerChunk;
   }
   auto load = [&](int64_t c, uint4* u) {
     const int total = chunk_tokens(c) * a.row_chunks;
@@ -287,39 +291,26 @@ __global__ void __launch_bounds__(kRopeThreads, 2) rope_bulk_kernel(const RopeBu
       rope_cos_sin(t, a.f.theta[p], cc, sn);
       step_tab[e] = make_float2(cc, sn);
     }
+  __syncthreads();
   int64_t c = blockIdx.x;
   if (c < n_chunks) prepare(c, 0);
   uint4 u[kRopePieces], un[kRopePieces];
   if (c < n_chunks) load(c, u);
   for (int i = 0; c < n_chunks; c += step, ++i) {
     const int buf = i & 1;
-    __syncthreads();                                  // angles of chunk c are in buffer buf
+    __syncthreads();                                  // the table of chunk c is in buffer buf
     const bool more = c + step < n_chunks;
     if (more) load(c + step, un);                     // next chunk's loads in flight during this one
-    int64_t n0;
-    const bool one = in_one_entry(c, n0);
     const int total = chunk_tokens(c) * a.row_chunks;
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.out) + c * a.tok_per_chunk * a.token_bytes);
-    const float2* base = base_tab + buf * kMaxPairs;
-    const float2* dtab = direct_tab(buf);
+    const float2* tab = chunk_tab(buf);
 #pragma unroll
     for (int k = 0; k < kRopePieces; ++k) {
       const int e = tid + k * kRopeThreads;
       if (e < total) {
         float2 cs[kPairsPerChunk];
-        const int t = pt[k], p0 = pp[k];
-        if (dense_pos && one) {
 #pragma unroll
-          for (int q = 0; q < kPairsPerChunk; ++q) cs[q] = cs_add(base[p0 + q], step_tab[t * pairs + p0 + q]);
-        } else if (!dense_pos) {
-#pragma unroll
-          for (int q = 0; q < kPairsPerChunk; ++q) cs[q] = dtab[t * pairs + p0 + q];
-        } else {
-          int64_t n = n0 + t;
-          while (n >= a.N) n -= a.N;
-#pragma unroll
-          for (int q = 0; q < kPairsPerChunk; ++q) rope_cos_sin(n, a.f.theta[p0 + q], cs[q].x, cs[q].y);
-        }
+        for (int q = 0; q < kPairsPerChunk; ++q) cs[q] = tab[pofs[k] + q];
         rope_chunk_regs<T>(u[k], cs);
         dst[e] = u[k];
       }

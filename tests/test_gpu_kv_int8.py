@@ -68,6 +68,21 @@ def test_quantize_strided_view():
     assert not out[:, :, 4].any()                          # nothing written outside the view
 
 
+def test_quantize_8_byte_rows_and_odd_row_count():
+    # bf16 rows 8- but not 16-byte aligned take the warp-per-row kernel; an odd
+    # number of rows exercises the last half-warp of the 16-byte kernel.
+    base = _cache(1, 301, 3, seed=61)
+    pad = torch.zeros(1, 301, 3, 132, dtype=torch.bfloat16, device=DEV)
+    pad[..., 4:] = base
+    x8 = pad[..., 4:]                                      # rows start 8 bytes into 264-byte rows
+    for x in (x8, base):
+        codes, scale = _lib.kv_quantize_int8(x)
+        torch.cuda.synchronize()
+        c_ref, s_ref = orc.quantize_kv_int8(base.float().cpu().numpy())
+        assert np.array_equal(codes.cpu().numpy(), c_ref)
+        assert np.array_equal(scale.cpu().numpy(), s_ref)
+
+
 def _oracle_decode(q, k, v, inv_freq, t, q_index, window, n_sink):
     """Oracle O [Hq, d], LSE [Hq] of one query token against an int8 cache of k, v.
 
