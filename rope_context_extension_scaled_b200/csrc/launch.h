@@ -14,7 +14,6 @@ namespace rcx {
 
 struct AttnArgs;
 struct RopeArgs;
-struct RopeBulkArgs;
 struct MergeArgs;
 struct DecodeArgs;
 struct QuantArgs;
@@ -46,8 +45,7 @@ inline int allow_smem(K kernel, size_t bytes) {
 }
 
 // ---- k_rope.cu
-int rope_bulk_launch(const RopeBulkArgs& b, int dtype, int grid, size_t smem, cudaStream_t stream);
-int rope_apply_launch(const RopeArgs& a, int dtype, bool same_layout, int grid, cudaStream_t stream);
+int rope_apply_launch(const RopeArgs& a, int dtype, int grid, int block, cudaStream_t stream);
 
 // ---- k_merge.cu
 int merge_launch(const MergeArgs& a, int out_dtype, int grid, cudaStream_t stream);

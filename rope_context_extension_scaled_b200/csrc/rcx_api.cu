@@ -212,69 +212,6 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   }
   if (positions && n_positions < N) return RCX_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return RCX_OK;
-  {
-    // Dense views (every token one contiguous row, in and out) take the
-    // bulk-copy kernel, one launch per operand.
-    auto dense = [](const rcx_tensor& t) {
-      return t.stride[3] == 1 && t.stride[2] == t.shape[3] && t.stride[1] == t.shape[2] * t.shape[3] &&
-             (t.shape[0] == 1 || t.stride[0] == t.shape[1] * t.stride[1]);
-    };
-    bool all_dense = true;
-    for (int i = 0; i < 2; ++i)
-      if (ins[i]->ptr) {
-        const int64_t tb = ins[i]->shape[2] * D * elem_size(dtype);
-        all_dense = all_dense && dense(*ins[i]) && dense(*outs[i]) && tb <= kRopeBulkBytes && tb % 16 == 0;
-      }
-    if (all_dense) {
-      const size_t smem = kRopeBulkSmem;
-      for (int i = 0; i < 2; ++i) {
-        if (!ins[i]->ptr) continue;
-        RopeBulkArgs b;
-        std::memset(&b, 0, sizeof(b));
-        b.in = ins[i]->ptr;
-        b.out = outs[i]->ptr;
-        b.positions = positions;
-        b.n_tok = B * N;
-        b.N = N;
-        b.d = (int)D;
-        b.pairs = (int)(D / 2);
-        b.token_bytes = ins[i]->shape[2] * D * elem_size(dtype);
-        b.tok_per_chunk = (int)std::max<int64_t>(
-            1, std::min<int64_t>(kRopeBulkBytes / b.token_bytes, kRopeBulkTab / b.pairs));
-        b.row_chunks = (int)(b.token_bytes / 16);
-        b.d_chunks = (int)(D * elem_size(dtype) / 16);
-        for (int j = 0; j < b.pairs; ++j) b.f.theta[j] = inv_freq[j];
-        const int64_t chunks = (b.n_tok + b.tok_per_chunk - 1) / b.tok_per_chunk;
-        const int grid = (int)std::min<int64_t>(chunks, (int64_t)sm_count() * 4);
-        const int st = rope_bulk_launch(b, dtype, grid, smem, stream);
-        if (st) return st;
-      }
-      return RCX_OK;
-    }
-  }
-  const int elems = 16 / elem_size(dtype);
-  const int64_t cph = D / elems;                      // 16-byte chunks per head
-  const int64_t max_chunks = (int64_t)kRopeSlots * kRopeThreads;
-  const int64_t cpt = ((has_q ? q.shape[2] : 0) + (has_k ? k.shape[2] : 0)) * cph;
-  if (cpt > max_chunks) {
-    // More chunks per token than one pass holds: rotate head ranges separately.
-    const int64_t hmax = std::max<int64_t>(1, max_chunks / cph);
-    for (int i = 0; i < 2; ++i) {
-      if (!ins[i]->ptr) continue;
-      for (int64_t h0 = 0; h0 < ins[i]->shape[2]; h0 += hmax) {
-        const int64_t nh = std::min(hmax, ins[i]->shape[2] - h0);
-        rcx_tensor si = *ins[i], so = *outs[i];
-        si.ptr = static_cast<char*>(si.ptr) + h0 * si.stride[2] * elem_size(dtype);
-        so.ptr = static_cast<char*>(so.ptr) + h0 * so.stride[2] * elem_size(dtype);
-        si.shape[2] = so.shape[2] = nh;
-        const rcx_tensor nul = null_tensor();
-        int st = i == 0 ? rope_apply_impl(si, nul, so, nul, positions, n_positions, inv_freq, stream)
-                        : rope_apply_impl(nul, si, nul, so, positions, n_positions, inv_freq, stream);
-        if (st) return st;
-      }
-    }
-    return RCX_OK;
-  }
   RopeArgs a;
   std::memset(&a, 0, sizeof(a));
   if (has_q) { a.q_in = make_view(q); a.q_out = make_view(q_out); }
@@ -282,16 +219,12 @@ int rope_apply_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& 
   a.positions = positions;
   a.n_tok = B * N;
   a.N = N;
-  a.pairs = (int)(D / 2);
-  int64_t tpi = std::min<int64_t>(kRopeMaxTok, std::max<int64_t>(1, max_chunks / cpt));
-  tpi = std::min<int64_t>(tpi, kRopeMaxAngles / a.pairs);
-  a.tok_per_iter = (int)std::max<int64_t>(1, tpi);
-  for (int i = 0; i < a.pairs; ++i) a.f.theta[i] = inv_freq[i];
-  const int64_t groups = (a.n_tok + a.tok_per_iter - 1) / a.tok_per_iter;
-  const int grid = (int)std::min<int64_t>(groups, (int64_t)sm_count() * 6);
-  auto same = [](const View4& x, const View4& y) { return x.sb == y.sb && x.sn == y.sn && x.sh == y.sh; };
-  const bool same_layout = (!has_q || same(a.q_in, a.q_out)) && (!has_k || same(a.k_in, a.k_out));
-  return rope_apply_launch(a, dtype, same_layout, grid, stream);
+  a.d_chunks = (int)(D * elem_size(dtype) / 16);    // vec16_ok: D * element size is a multiple of 16
+  for (int i = 0; i < (int)(D / 2); ++i) a.f.theta[i] = inv_freq[i];
+  const int tpb = kRopeThreads / a.d_chunks;          // d_chunks <= 2 * kMaxPairs * 4 / 16 = 64
+  const int64_t passes = (a.n_tok + tpb - 1) / tpb;
+  const int grid = (int)std::min<int64_t>(passes, (int64_t)sm_count() * kRopeCtasPerSm);
+  return rope_apply_launch(a, dtype, grid, tpb * a.d_chunks, stream);
 }
 
 // ---------------------------------------------------------------------- merge

@@ -87,14 +87,14 @@ def test_rope_angle_error_at_one_million():
 
 
 @pytest.mark.parametrize("d", [128, 64])
-def test_rope_bulk_path_angle_error_near_one_million(d):
-    # Dense layout and positions == NULL take the bulk-copy kernel, whose
-    # angles for consecutive tokens come from an exact per-chunk base angle
-    # and an exact step angle (angle-addition identity).  Unit vectors (1, 0)
-    # in every pair, fp32, N = 2^20 tokens of one head (chunks of 16 tokens at
-    # d = 128, 32 at d = 64): the applied angle of every pair must be within
-    # 1e-5 rad of m * theta' (60-digit arithmetic), including chunks that start
-    # just below m = 1,048,575 and every offset within a chunk.
+def test_rope_dense_angle_error_near_one_million(d):
+    # Dense layout, positions == NULL (position = token index), fp32 unit
+    # vectors (1, 0) in every pair, N = 2^20 tokens of one head: the applied
+    # angle of every pair must be within 1e-5 rad of m * theta' (40-digit
+    # arithmetic), for the last 192 tokens below m = 1,048,575, the first 40
+    # and 96 random ones.  Each token's angles are computed on their own
+    # (float64 product and reduction, fp32 sincos), so the bound that holds is
+    # the one of a single sincos: 2e-6.
     N = 1 << 20
     inv, _, _, _ = schedule(_lib.NTK, 5e5, d, 8192, 1 << 20)
     x = torch.zeros(1, N, 1, d, dtype=torch.float32, device=DEV)
@@ -115,8 +115,42 @@ def test_rope_bulk_path_angle_error_near_one_million(d):
             ex = float(e - two_pi * mpmath.nint(e / two_pi))
             diff = abs((got[r, i] - ex + math.pi) % (2 * math.pi) - math.pi)
             worst = max(worst, diff)
-    print(f"bulk rope_apply d={d}: worst angle error {worst:.3e} rad over {len(toks)} tokens")
+    print(f"dense rope_apply d={d}: worst angle error {worst:.3e} rad over {len(toks)} tokens")
     assert worst <= 1e-5, worst
+    assert worst <= 2e-6, worst
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 96), (torch.bfloat16, 8), (torch.float32, 256),
+                                     (torch.float32, 4), (torch.bfloat16, 128)])
+def test_rope_apply_strided_views_and_odd_widths(dtype, d):
+    # Q and K as head slices of one packed [B, N, Hq + 2 Hkv, d] tensor (row
+    # stride != H * d), outputs into [B, H, N, d] storage seen as [B, N, H, d]
+    # (head stride N * d); Hq + Hkv = 11 heads, so one thread's group of heads
+    # straddles the Q/K boundary; head widths whose 16-byte pieces per head
+    # (12, 1, 64, 1, 16) give CTAs of 252, 256, 256, 256 and 256 threads.
+    B, N, Hq, Hkv = 3, 45, 8, 3
+    g = torch.Generator(device="cpu")
+    g.manual_seed(41)
+    qkv = torch.randn(B, N, Hq + 2 * Hkv, d, generator=g).to(dtype).to(DEV)
+    q, k = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv]
+    qo = torch.empty(B, Hq, N, d, dtype=dtype, device=DEV).transpose(1, 2)
+    ko = torch.empty(B, Hkv, N, d, dtype=dtype, device=DEV).transpose(1, 2)
+    inv, _, oinv, _ = schedule(_lib.YARN, 1e4, d, 4096, 65536)
+    pos = torch.randint(0, 1 << 17, (N,), generator=g, dtype=torch.int64).to(DEV)
+    v_before = qkv[:, :, Hq + Hkv:].clone()
+    _lib.rope_apply(q, k, inv, positions=pos, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    p_np = pos.cpu().numpy()
+    for x, y in ((q, qo), (k, ko)):
+        for b in range(B):
+            ref = orc.rope_rotate(np64(x[b]), p_np, oinv)
+            got = np64(y[b])
+            if dtype == torch.float32:
+                assert np.abs(got - ref).max() < 1e-5
+            else:
+                assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5)
+    # the V slice of the packed tensor is not written
+    assert torch.equal(qkv[:, :, Hq + Hkv:], v_before)
 
 
 def test_rope_apply_rejects_misaligned():
@@ -490,7 +524,7 @@ def test_ring_batch2(dtype, d):
 
 
 def test_rope_apply_batch_wrap_in_chunk():
-    # N smaller than a bulk chunk: chunks straddle batch entries (direct angles).
+    # N smaller than a CTA's pass of tokens: one pass covers several batch entries.
     B, N = 5, 3
     q, k, _ = make_qkv(B, N, 2, 8, 128, torch.bfloat16, seed=32, device=DEV)
     inv, _, oinv, _ = schedule(_lib.PLAIN, 1e4, 128, 10, 10)
