@@ -43,6 +43,11 @@ WORKLOADS = {
                                       131072, window=4096, n_sink=4, sample_rows=4096),
     "llama3_70b_1m_ring": Workload("llama3_70b_1m_ring", 1, 64, 8, 128, 1 << 20, "bf16", NTK, 5e5, 8192, 1 << 20,
                                    kv_block=65536, ring=True, sample_rows=4096),
+    # Three ring blocks of the 1M workload's shape (65,536 keys, same heads and
+    # schedule): every launch form of the 1M ring (direct bf16 output, first,
+    # middle and last partial) at 196,608 tokens, small enough to profile.
+    "llama3_70b_192k_ring": Workload("llama3_70b_192k_ring", 1, 64, 8, 128, 3 * 65536, "bf16", NTK, 5e5, 8192,
+                                     1 << 20, kv_block=65536, ring=True, sample_rows=4096),
     "llama3_8b_128k_ring": Workload("llama3_8b_128k_ring", 1, 32, 8, 128, 131072, "bf16", NTK, 5e5, 8192, 131072,
                                     kv_block=32768, ring=True, sample_rows=4096),
 }

@@ -50,7 +50,7 @@ int decode_combine_launch(const DecodeArgs& a, int out_dtype, int grid, cudaStre
 int quantize_i8_launch(const QuantArgs& a, bool rows16, int grid, cudaStream_t stream) {
   LaunchScope scope(RCX_KERNEL_DECODE, stream);
   if (rows16)
-    kv_quantize_int8_h16_kernel<<<grid, 256, 0, stream>>>(a);
+    kv_quantize_int8_r8_kernel<<<grid, 256, 0, stream>>>(a);
   else
     kv_quantize_int8_kernel<<<grid, 256, 0, stream>>>(a);
   return launch_status();

@@ -44,6 +44,7 @@ struct QuantArgs {
   View4 c;          // int8 [B, N, H, 128]
   float* scale;     // [B, N, H] contiguous
   int64_t rows;     // B * N * H
+  int dense;        // x and c are [rows, 128] with no gaps: row r starts at r * 128
 };
 
 // One warp per row; lane l holds dims 4l .. 4l + 3.  A warp takes kQRows rows
@@ -101,16 +102,36 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const Quan
   }
 }
 
-// Half-warp per row, for rows whose bf16 values and codes are 16- and 8-byte
-// aligned: lane l of a half holds dims 8l .. 8l + 7 (one 16-byte load, so a
-// row is one coalesced 256-byte read), the row max takes four shuffles within
-// the half, and each lane stores its 8 codes as one 8-byte word.  A warp has
-// kQRowsH row pairs in flight per pass, all loads issued before any
-// arithmetic.  Same IEEE fp32 decisions as kv_quantize_int8_kernel, so the
-// codes and scales are identical.
-constexpr int kQRowsH = 4;
+// Eight lanes per row, for rows whose bf16 values and codes are both 16-byte
+// aligned: lane l of an eight-lane group holds dims 16l .. 16l + 15 (two
+// 16-byte loads, so a row is one coalesced 256-byte read), the row max takes
+// three shuffles within the group, and the lane stores its 16 codes as one
+// 16-byte word.  A warp covers four rows per pass and keeps kQPasses passes of
+// loads in flight.  The per-row work (max, the two IEEE divisions, the row
+// offsets) is shared by 16 values per lane, which keeps the kernel below the
+// SM's issue rate at HBM speed.  Rounding: y = fl(x * inv) satisfies |y| <= 127
+// (inv = fl(127 / amax) exceeds 127 / amax by at most half an ulp, so
+// |y| < 127.5 and rint(y) is within [-127, 127], where the clamp never acts),
+// and fl(y + 1.5 * 2^23) holds rint(y), ties to even, in its low bits (the sum
+// lies in [2^23, 2^24), where the fp32 spacing is 1), whose low byte is the
+// two's-complement code.  So the codes and scales equal those of
+// kv_quantize_int8_kernel.
+constexpr int kQPasses = 2;
+
+__device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float inv) {
+  const float kRound = 12582912.f;                      // 1.5 * 2^23
+  const uint32_t qa = __float_as_uint(__fadd_rn(__fmul_rn(a, inv), kRound));
+  const uint32_t qb = __float_as_uint(__fadd_rn(__fmul_rn(b, inv), kRound));
+  const uint32_t qc = __float_as_uint(__fadd_rn(__fmul_rn(c, inv), kRound));
+  const uint32_t qd = __float_as_uint(__fadd_rn(__fmul_rn(d, inv), kRound));
+  return __byte_perm(__byte_perm(qa, qb, 0x0040), __byte_perm(qc, qd, 0x0040), 0x5410);
+}
 
 __device__ __forceinline__ void quant_row_offsets(const QuantArgs& a, int64_t r, int64_t& off_x, int64_t& off_c) {
+  if (a.dense) {                              // [rows, 128] in both: no index decoding
+    off_x = off_c = r * 128;
+    return;
+  }
   int64_t h, n, b;
   if (a.rows < (int64_t(1) << 31)) {          // 32-bit index arithmetic (the usual case)
     const uint32_t r32 = (uint32_t)r, H32 = (uint32_t)a.x.H, N32 = (uint32_t)a.x.N;
@@ -127,47 +148,56 @@ __device__ __forceinline__ void quant_row_offsets(const QuantArgs& a, int64_t r,
   off_c = b * a.c.sb + n * a.c.sn + h * a.c.sh;
 }
 
-static __global__ void __launch_bounds__(256) kv_quantize_int8_h16_kernel(const QuantArgs a) {
+static __global__ void __launch_bounds__(256) kv_quantize_int8_r8_kernel(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4, hl = lane & 15;
-  const int64_t pairs = (a.rows + 1) / 2;
+  const int sub = lane >> 3, el = lane & 7;
+  const int64_t quads = (a.rows + 3) / 4;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
   const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  for (int64_t p0 = w0; p0 < pairs; p0 += kQRowsH * nwarps) {
-    uint4 u[kQRowsH];
-    int64_t off_c[kQRowsH];
+  for (int64_t p0 = w0; p0 < quads; p0 += kQPasses * nwarps) {
+    uint4 u[kQPasses][2];
+    int64_t off_c[kQPasses];
 #pragma unroll
-    for (int i = 0; i < kQRowsH; ++i) {
+    for (int i = 0; i < kQPasses; ++i) {
       const int64_t p = p0 + i * nwarps;
-      int64_t r = 2 * (p < pairs ? p : p0) + half;
-      if (r >= a.rows) r = a.rows - 1;               // odd row count: the last half repeats a row, stores nothing
+      int64_t r = 4 * (p < quads ? p : p0) + sub;
+      if (r >= a.rows) r = a.rows - 1;               // ragged last quad: repeats a row, stores nothing
       int64_t off_x;
       quant_row_offsets(a, r, off_x, off_c[i]);
-      u[i] = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.x.ptr) + off_x + 8 * hl);
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.x.ptr) + off_x) + 2 * el;
+      u[i][0] = __ldcs(src);
+      u[i][1] = __ldcs(src + 1);
     }
 #pragma unroll
-    for (int i = 0; i < kQRowsH; ++i) {
+    for (int i = 0; i < kQPasses; ++i) {
       const int64_t p = p0 + i * nwarps;
-      if (p >= pairs) break;                         // warp-uniform
-      const int64_t r = 2 * p + half;
-      const float2 x01 = bf2_to_f2(u[i].x), x23 = bf2_to_f2(u[i].y), x45 = bf2_to_f2(u[i].z), x67 = bf2_to_f2(u[i].w);
-      const float v[8] = {x01.x, x01.y, x23.x, x23.y, x45.x, x45.y, x67.x, x67.y};
+      if (p >= quads) break;                         // warp-uniform
+      const int64_t r = 4 * p + sub;
+      float v[16];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t w[4] = {u[i][h].x, u[i][h].y, u[i][h].z, u[i][h].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = bf2_to_f2(w[e]);
+          v[8 * h + 2 * e] = f.x;
+          v[8 * h + 2 * e + 1] = f.y;
+        }
+      }
       float am = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
+      for (int e = 0; e < 16; ++e) am = fmaxf(am, fabsf(v[e]));
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+      for (int off = 4; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
       const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
-      uint32_t w[2] = {0u, 0u};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        int q = __float2int_rn(__fmul_rn(v[e], inv));
-        q = q > 127 ? 127 : (q < -127 ? -127 : q);
-        w[e >> 2] |= (uint32_t)(q & 0xff) << (8 * (e & 3));
-      }
+      uint4 q;
+      q.x = quant4(v[0], v[1], v[2], v[3], inv);
+      q.y = quant4(v[4], v[5], v[6], v[7], inv);
+      q.z = quant4(v[8], v[9], v[10], v[11], inv);
+      q.w = quant4(v[12], v[13], v[14], v[15], inv);
       if (r < a.rows) {
-        *reinterpret_cast<uint2*>(reinterpret_cast<int8_t*>(a.c.ptr) + off_c[i] + 8 * hl) = make_uint2(w[0], w[1]);
-        if (hl == 0) a.scale[r] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
+        *reinterpret_cast<uint4*>(reinterpret_cast<int8_t*>(a.c.ptr) + off_c[i] + 16 * el) = q;
+        if (el == 0) a.scale[r] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
       }
     }
   }
@@ -352,21 +382,23 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
       kw[r][0] = u0.x; kw[r][1] = u0.y; kw[r][2] = u0.z; kw[r][3] = u0.w;
       kw[r][4] = u1.x; kw[r][5] = u1.y; kw[r][6] = u1.z; kw[r][7] = u1.w;
     }
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    // two accumulator chains (even and odd k chunks) halve the dependent MMA sequence
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kc = 0; kc < 8; ++kc) {
       const uint32_t fa = kw[0][kc] ^ 0x80808080u, fb = kw[1][kc] ^ 0x80808080u;
       const uint32_t af[4] = {codes_to_h2_off(fa, 0x4140), codes_to_h2_off(fb, 0x4140), codes_to_h2_off(fa, 0x4342),
                               codes_to_h2_off(fb, 0x4342)};
-      mma_f16_16816(sacc, af, qb[kc][0], qb[kc][1]);
+      mma_f16_16816((kc & 1) ? sacc2 : sacc, af, qb[kc][0], qb[kc][1]);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
     // key scales, online softmax per head over keys t0 + g, t0 + g + 8
     const float ska = sk[g], skb = sk[g + 8];
     const float sva = sv_[g], svb = sv_[g + 8];
-    float tmax = fmaxf(sva, svb);
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+    // largest V scale of the tile: scales are >= 0, so their bit patterns order
+    // like the values and one integer max-reduction over the warp finds it
+    const float tmax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(sva, svb))));
     const float smax_new = fmaxf(smax, tmax);
     const float ratio = smax_new > 0.f ? smax / smax_new : 1.f;
     const float inv_smax = smax_new > 0.f ? 1.f / smax_new : 0.f;
@@ -406,12 +438,18 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
       const int key = 2 * c + (i & 1) + 8 * (i >> 1);
       vr[i] = *reinterpret_cast<const uint4*>(vs + key * kDqRow + 16 * g);
     }
+    // O rescale only when some column's factor moved (the max or s_max grew)
+    if (__any_sync(0xffffffffu, beta[0] != 1.f || beta[1] != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        o[mt][0] *= beta[0];
+        o[mt][1] *= beta[1];
+        o[mt][2] *= beta[0];
+        o[mt][3] *= beta[1];
+      }
+    }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      o[mt][0] *= beta[0];
-      o[mt][1] *= beta[1];
-      o[mt][2] *= beta[0];
-      o[mt][3] *= beta[1];
       // operand rows: dim 16g + 2mt (row g) and 16g + 2mt + 1 (row g + 8)
       const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;   // bytes j, j + 1 of two keys, interleaved
       const int wi = mt >> 1;

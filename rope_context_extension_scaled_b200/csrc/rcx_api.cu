@@ -447,12 +447,18 @@ int quantize_i8_impl(const rcx_tensor& x, const rcx_tensor& c, float* scale, cud
   if (!scale) return RCX_ERR_INVALID_ARG;
   if (!aligned_rows(x, 8) || !aligned_rows(c, 4) || reinterpret_cast<uintptr_t>(scale) % 4) return RCX_ERR_ALIGNMENT;
   QuantArgs a;
+  std::memset(&a, 0, sizeof(a));
   a.x = make_view(x);
   a.c = make_view(c);
   a.scale = scale;
   a.rows = rows;
-  const bool rows16 = aligned_rows(x, 16) && aligned_rows(c, 8);
-  const int64_t per_cta = rows16 ? 16 : 8;      // rows a CTA covers per pass (two or one per warp)
+  auto packed = [](const rcx_tensor& t) {     // [B, N, H, 128] with no gaps
+    return t.stride[3] == 1 && t.stride[2] == 128 && t.stride[1] == t.shape[2] * 128 &&
+           (t.shape[0] == 1 || t.stride[0] == t.shape[1] * t.stride[1]);
+  };
+  a.dense = packed(x) && packed(c);
+  const bool rows16 = aligned_rows(x, 16) && aligned_rows(c, 16);
+  const int64_t per_cta = rows16 ? 32 : 8;      // rows a CTA covers per pass (four or one per warp)
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + per_cta - 1) / per_cta,
                                                               (int64_t)sm_count() * 8));
   return quantize_i8_launch(a, rows16, grid, stream);

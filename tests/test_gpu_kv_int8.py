@@ -69,8 +69,9 @@ def test_quantize_strided_view():
 
 
 def test_quantize_8_byte_rows_and_odd_row_count():
-    # bf16 rows 8- but not 16-byte aligned take the warp-per-row kernel; an odd
-    # number of rows exercises the last half-warp of the 16-byte kernel.
+    # bf16 rows 8- but not 16-byte aligned take the warp-per-row kernel; 903
+    # rows (not a multiple of four) exercise the ragged last group of four rows
+    # of the 16-byte kernel.
     base = _cache(1, 301, 3, seed=61)
     pad = torch.zeros(1, 301, 3, 132, dtype=torch.bfloat16, device=DEV)
     pad[..., 4:] = base
