@@ -224,8 +224,9 @@ int rcx_attn_decode_fwd(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, 
  * same bytes.
  *
  * x: [B, N, H, 128] bf16, 8-byte aligned rows.  codes: [B, N, H, 128]
- * RCX_I8, same shape, 4-byte aligned rows.  scale: device fp32 [B, N, H],
- * contiguous (row (b, n, h) at (b * N + n) * H + h), caller-owned.  Memory
+ * RCX_I8, same shape, 4-byte aligned rows.  scale: device fp32 [B, H, N],
+ * contiguous and head-major (row (b, n, h) at (b * H + h) * N + n, so one
+ * head's scales for consecutive tokens are adjacent), caller-owned.  Memory
  * bound: reads x once, writes codes and scales once.  Launches are timed
  * under RCX_KERNEL_DECODE.
  */
@@ -234,7 +235,7 @@ int rcx_kv_quantize_int8(rcx_tensor x, rcx_tensor codes, float* scale, void* str
 /*
  * rcx_attn_decode_int8_fwd -- rcx_attn_decode_fwd over an int8 KV cache made
  * by rcx_kv_quantize_int8: key j of KV head h stands for k_codes[j] *
- * k_scale[j, h] (and likewise V).  Same query, mask, GQA, temperature, LSE,
+ * k_scale[h, j] (and likewise V).  Same query, mask, GQA, temperature, LSE,
  * rope_flags and split-KV merge as rcx_attn_decode_fwd; the codes are
  * dequantised in the tile load and the contractions run in fp16 with fp32
  * accumulation, so |rotated q| and the dequantised V must stay below the fp16
@@ -242,7 +243,8 @@ int rcx_kv_quantize_int8(rcx_tensor x, rcx_tensor codes, float* scale, void* str
  *
  * q, o: [B, 1, Hq, 128] (q bf16; o bf16 or f32); k, v: [B, Nk, Hkv, 128]
  * RCX_I8, 16-byte aligned rows (base and strides multiples of 16 bytes);
- * k_scale, v_scale: device fp32 [B, Nk, Hkv] contiguous; Hq / Hkv in
+ * k_scale, v_scale: device fp32 [B, Hkv, Nk] contiguous (the layout
+ * rcx_kv_quantize_int8 writes); Hq / Hkv in
  * {1, 2, 4, 8}; lse: [B, Hq, 1, 1] fp32 or ptr NULL.  workspace: device
  * buffer of rcx_attn_decode_int8_workspace_size(q, k) bytes, 256-byte
  * aligned, caller-owned.  Memory-bound: reads each code and scale once (half

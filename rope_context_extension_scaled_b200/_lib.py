@@ -331,14 +331,14 @@ def ring_attn_fwd_noalloc(q, k, v, o, lse=None, kv_block=0, window=0, n_sink=0, 
 
 
 def kv_quantize_int8(x, codes=None, scale=None):
-    """Int8 codes [B, N, H, 128] and fp32 scales [B, N, H] of a bf16 cache x."""
+    """Int8 codes [B, N, H, 128] and fp32 scales [B, H, N] (head-major) of a bf16 cache x."""
     B, N, H, _ = x.shape
     if codes is None:
         codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
     if scale is None:
-        scale = torch.empty(B, N, H, dtype=torch.float32, device=x.device)
-    if not scale.is_contiguous() or scale.dtype != torch.float32 or tuple(scale.shape) != (B, N, H):
-        raise ValueError("scale must be a contiguous float32 [B, N, H] tensor")
+        scale = torch.empty(B, H, N, dtype=torch.float32, device=x.device)
+    if not scale.is_contiguous() or scale.dtype != torch.float32 or tuple(scale.shape) != (B, H, N):
+        raise ValueError("scale must be a contiguous float32 [B, H, N] tensor")
     st = load().rcx_kv_quantize_int8(view(x), view(codes), ctypes.c_void_p(scale.data_ptr()), _stream(x.device))
     _check(st, "rcx_kv_quantize_int8")
     return codes, scale
@@ -346,7 +346,7 @@ def kv_quantize_int8(x, codes=None, scale=None):
 
 def attn_decode_int8_fwd(q, k, k_scale, v, v_scale, o=None, lse=None, window=0, n_sink=0, temperature=1.0,
                          q_index=None, positions=None, inv_freq=None, rope_flags=0, workspace=None, want_lse=True):
-    """attn_decode_fwd over an int8 cache (codes k, v [B, Nk, Hkv, 128], scales [B, Nk, Hkv])."""
+    """attn_decode_fwd over an int8 cache (codes k, v [B, Nk, Hkv, 128], scales [B, Hkv, Nk])."""
     B, _, H, D = q.shape
     if q_index is None:
         q_index = k.shape[1] - 1
@@ -354,9 +354,10 @@ def attn_decode_int8_fwd(q, k, k_scale, v, v_scale, o=None, lse=None, window=0, 
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, H, 1, dtype=torch.float32, device=q.device)
+    Bk, Nk, Hkv = k.shape[:3]
     for sc in (k_scale, v_scale):
-        if not sc.is_contiguous() or sc.dtype != torch.float32 or tuple(sc.shape) != tuple(k.shape[:3]):
-            raise ValueError("scales must be contiguous float32 [B, Nk, Hkv] tensors")
+        if not sc.is_contiguous() or sc.dtype != torch.float32 or tuple(sc.shape) != (Bk, Hkv, Nk):
+            raise ValueError("scales must be contiguous float32 [B, Hkv, Nk] tensors")
     need = load().rcx_attn_decode_int8_workspace_size(view(q), view(k))
     if need < 0:
         raise RcxError(RCX_ERR_INVALID_ARG, "rcx_attn_decode_int8_workspace_size")

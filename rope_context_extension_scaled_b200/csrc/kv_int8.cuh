@@ -6,10 +6,14 @@
 // (the plainest symmetric reading; the pages fix none): one fp32 scale per
 // row of d = 128 values (one token of one KV head), scale = amax / 127 and
 // code = rint(x * (127 / amax)) in [-127, 127], all decided in IEEE fp32.
+// Scales are stored head-major, [B, H, N], so that the scales of a tile of
+// consecutive keys of one head are one contiguous row.
 //
-// Decode over the codes follows attn_decode_mma_kernel (16-key tiles per
-// warp, three cp.async stages, transposed mma.sync with the G <= 8 query heads
-// as the MMA columns) with the dequantisation in the tile load:
+// Decode over the codes follows attn_decode_mma_kernel (three cp.async stages
+// per warp, transposed mma.sync with the G <= 8 query heads as the MMA
+// columns), with 32-key tiles so that a tile moves as many bytes as the bf16
+// kernel's 16-key tile and the per-tile softmax work is shared by 32 keys, and
+// the dequantisation in the tile load:
 //  * the MMAs run in fp16 (m16n8k16, fp32 accumulate), because an int8 code
 //    becomes an exact fp16 in three integer/half instructions: the byte with
 //    its sign bit flipped (u = code + 128) is placed under the exponent
@@ -29,8 +33,12 @@
 // K row reads use the same d permutation trick as the bf16 kernel's first
 // form: lane c of a row group takes dims [32c, 32c + 32) of the key in order,
 // and Q is laid out with the same permutation, so every dot product is
-// unchanged.  The V^T operand rows (d) are permuted too: lane g's rows are
-// dims [16g, 16g + 16), and the merge writes them back in natural order.
+// unchanged.  The V^T operand comes from ldmatrix.trans of the code tile read
+// as 16-bit elements (two dims of one key), which hands each lane dims 2g and
+// 2g + 1 of two consecutive keys in one register: A row g of m-tile mt is dim
+// 16 mt + 2g and row g + 8 is dim 16 mt + 2g + 1, so each register becomes two
+// A registers by two byte selections, and the merge writes the rows back in
+// natural order.
 #pragma once
 #include <cuda_fp16.h>
 #include "attn_decode.cuh"
@@ -39,12 +47,35 @@ namespace rcx {
 
 // ---------------------------------------------------------------- quantise
 
+// Unsigned division by a run-time constant d, exact for n < 2^31 (Granlund
+// and Montgomery, "Division by invariant integers using multiplication",
+// 1994): with l = ceil(log2 d), p = 31 + l and m = ceil(2^p / d) (< 2^32),
+// floor(n / d) = (n * m) >> p, because m = (2^p + e) / d with 0 <= e < d adds
+// n e / (d 2^p) < 2^(31 - p) <= 1 / d to n / d.
+struct FastDiv {
+  uint32_t m, p;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((uint64_t(1) << l) < d) ++l;
+  FastDiv f;
+  f.p = 31 + l;
+  f.m = (uint32_t)(((uint64_t(1) << f.p) + d - 1) / d);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
+  return (uint32_t)(((uint64_t)n * f.m) >> f.p);
+}
+
 struct QuantArgs {
   View4 x;          // bf16 [B, N, H, 128]
   View4 c;          // int8 [B, N, H, 128]
-  float* scale;     // [B, N, H] contiguous
+  float* scale;     // [B, H, N] contiguous (head-major)
   int64_t rows;     // B * N * H
-  int dense;        // x and c are [rows, 128] with no gaps: row r starts at r * 128
+  FastDiv div_h, div_n;    // by H and by N, exact for rows < 2^31
+  int fast;         // rows < 2^31: 32-bit row decoding by div_h / div_n
 };
 
 // One warp per row; lane l holds dims 4l .. 4l + 3.  A warp takes kQRows rows
@@ -57,7 +88,7 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const Quan
   const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   for (int64_t r0 = w0; r0 < a.rows; r0 += kQRows * nwarps) {
     uint2 u[kQRows];
-    int64_t off_c[kQRows];
+    int64_t off_c[kQRows], sidx[kQRows];
 #pragma unroll
     for (int i = 0; i < kQRows; ++i) {
       const int64_t r = r0 + i * nwarps;
@@ -78,6 +109,7 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const Quan
                                 h * a.x.sh + 4 * lane;
       u[i] = *reinterpret_cast<const uint2*>(xp);
       off_c[i] = b * a.c.sb + n * a.c.sn + h * a.c.sh + 4 * lane;
+      sidx[i] = (b * a.x.H + h) * a.x.N + n;
     }
 #pragma unroll
     for (int i = 0; i < kQRows; ++i) {
@@ -97,7 +129,7 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const Quan
         packed |= (uint32_t)(q & 0xff) << (8 * e);
       }
       *reinterpret_cast<uint32_t*>(reinterpret_cast<int8_t*>(a.c.ptr) + off_c[i]) = packed;
-      if (lane == 0) a.scale[r] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
+      if (lane == 0) a.scale[sidx[i]] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
     }
   }
 }
@@ -106,10 +138,11 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_kernel(const Quan
 // aligned: lane l of an eight-lane group holds dims 16l .. 16l + 15 (two
 // 16-byte loads, so a row is one coalesced 256-byte read), the row max takes
 // three shuffles within the group, and the lane stores its 16 codes as one
-// 16-byte word.  A warp covers four rows per pass and keeps kQPasses passes of
-// loads in flight.  The per-row work (max, the two IEEE divisions, the row
-// offsets) is shared by 16 values per lane, which keeps the kernel below the
-// SM's issue rate at HBM speed.  Rounding: y = fl(x * inv) satisfies |y| <= 127
+// 16-byte word.  A warp covers four consecutive rows (in [B, N, H] order) per
+// pass and keeps kQPasses passes of loads in flight.  The per-row work (max,
+// the two IEEE divisions, the row decoding by multiplicative division) is
+// shared by 16 values per lane, which keeps the kernel below the SM's issue
+// rate at HBM speed.  Rounding: y = fl(x * inv) satisfies |y| <= 127
 // (inv = fl(127 / amax) exceeds 127 / amax by at most half an ulp, so
 // |y| < 127.5 and rint(y) is within [-127, 127], where the clamp never acts),
 // and fl(y + 1.5 * 2^23) holds rint(y), ties to even, in its low bits (the sum
@@ -127,43 +160,39 @@ __device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, f
   return __byte_perm(__byte_perm(qa, qb, 0x0040), __byte_perm(qc, qd, 0x0040), 0x5410);
 }
 
-__device__ __forceinline__ void quant_row_offsets(const QuantArgs& a, int64_t r, int64_t& off_x, int64_t& off_c) {
-  if (a.dense) {                              // [rows, 128] in both: no index decoding
-    off_x = off_c = r * 128;
-    return;
-  }
-  int64_t h, n, b;
-  if (a.rows < (int64_t(1) << 31)) {          // 32-bit index arithmetic (the usual case)
-    const uint32_t r32 = (uint32_t)r, H32 = (uint32_t)a.x.H, N32 = (uint32_t)a.x.N;
-    const uint32_t t32 = r32 / H32;
-    h = r32 - t32 * H32;
-    n = t32 % N32;
-    b = t32 / N32;
-  } else {
-    h = r % a.x.H;
-    n = (r / a.x.H) % a.x.N;
-    b = r / (a.x.H * a.x.N);
-  }
-  off_x = b * a.x.sb + n * a.x.sn + h * a.x.sh;
-  off_c = b * a.c.sb + n * a.c.sn + h * a.c.sh;
-}
-
 static __global__ void __launch_bounds__(256) kv_quantize_int8_r8_kernel(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
   const int sub = lane >> 3, el = lane & 7;
   const int64_t quads = (a.rows + 3) / 4;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
   const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int64_t N = a.x.N, H = a.x.H;
   for (int64_t p0 = w0; p0 < quads; p0 += kQPasses * nwarps) {
     uint4 u[kQPasses][2];
-    int64_t off_c[kQPasses];
+    int64_t off_c[kQPasses], sidx[kQPasses];
+    bool live[kQPasses];
 #pragma unroll
     for (int i = 0; i < kQPasses; ++i) {
       const int64_t p = p0 + i * nwarps;
-      int64_t r = 4 * (p < quads ? p : p0) + sub;
-      if (r >= a.rows) r = a.rows - 1;               // ragged last quad: repeats a row, stores nothing
-      int64_t off_x;
-      quant_row_offsets(a, r, off_x, off_c[i]);
+      const int64_t r = 4 * (p < quads ? p : p0) + sub;   // row (b * N + n) * H + h
+      live[i] = p < quads && r < a.rows;                   // ragged last quad: repeats a row, stores nothing
+      const int64_t rr = r < a.rows ? r : a.rows - 1;
+      int64_t b, n, h;
+      if (a.fast) {
+        const uint32_t r32 = (uint32_t)rr;
+        const uint32_t t = fast_div(r32, a.div_h);
+        h = r32 - t * (uint32_t)H;
+        const uint32_t bb = fast_div(t, a.div_n);
+        n = t - bb * (uint32_t)N;
+        b = bb;
+      } else {
+        h = rr % H;
+        n = (rr / H) % N;
+        b = rr / (H * N);
+      }
+      const int64_t off_x = b * a.x.sb + n * a.x.sn + h * a.x.sh;
+      off_c[i] = b * a.c.sb + n * a.c.sn + h * a.c.sh;
+      sidx[i] = (b * H + h) * N + n;
       const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.x.ptr) + off_x) + 2 * el;
       u[i][0] = __ldcs(src);
       u[i][1] = __ldcs(src + 1);
@@ -172,16 +201,15 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_r8_kernel(const Q
     for (int i = 0; i < kQPasses; ++i) {
       const int64_t p = p0 + i * nwarps;
       if (p >= quads) break;                         // warp-uniform
-      const int64_t r = 4 * p + sub;
       float v[16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t w[4] = {u[i][h].x, u[i][h].y, u[i][h].z, u[i][h].w};
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t w[4] = {u[i][hf].x, u[i][hf].y, u[i][hf].z, u[i][hf].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = bf2_to_f2(w[e]);
-          v[8 * h + 2 * e] = f.x;
-          v[8 * h + 2 * e + 1] = f.y;
+          v[8 * hf + 2 * e] = f.x;
+          v[8 * hf + 2 * e + 1] = f.y;
         }
       }
       float am = 0.f;
@@ -195,9 +223,9 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_r8_kernel(const Q
       q.y = quant4(v[4], v[5], v[6], v[7], inv);
       q.z = quant4(v[8], v[9], v[10], v[11], inv);
       q.w = quant4(v[12], v[13], v[14], v[15], inv);
-      if (r < a.rows) {
+      if (live[i]) {
         *reinterpret_cast<uint4*>(reinterpret_cast<int8_t*>(a.c.ptr) + off_c[i] + 16 * el) = q;
-        if (el == 0) a.scale[r] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
+        if (el == 0) a.scale[sidx[i]] = am > 0.f ? __fdiv_rn(am, 127.f) : 0.f;
       }
     }
   }
@@ -205,12 +233,13 @@ static __global__ void __launch_bounds__(256) kv_quantize_int8_r8_kernel(const Q
 
 // ---------------------------------------------------------------- decode
 
-constexpr int kDqWarps = 8;
+constexpr int kDqWarps = 4;
 constexpr int kDqStages = 3;
+constexpr int kDqKeys = 32;                                  // keys per tile (two 16-key MMA halves)
 constexpr int kDqRow = 144;                                  // 128-byte code row + 16 pad (banks)
-constexpr int kDqTile = 16 * kDqRow;                         // one 16-key K or V tile
-constexpr int kDqStage = 2 * kDqTile + 2 * 64;               // K, V, 16 K scales, 16 V scales
-constexpr int kDqSmem = kDqWarps * kDqStages * kDqStage;     // 113,664 B: two CTAs (16 warps) per SM
+constexpr int kDqTile = kDqKeys * kDqRow;                    // one 32-key K or V tile
+constexpr int kDqStage = 2 * kDqTile + 2 * 4 * kDqKeys;      // K, V, 32 K scales, 32 V scales
+constexpr int kDqSmem = kDqWarps * kDqStages * kDqStage;     // 113,664 B: two CTAs (8 warps) per SM
 constexpr int kDqCtasPerSm = 2;
 static_assert(kDqSmem >= kDqWarps * kDecMaxG * 128 * 4, "merge area aliases the stage buffers");
 
@@ -296,55 +325,77 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
     qs[1] = __shfl_sync(0xffffffffu, part, 8 * c + 4) * 1152.f;
   }
 
-  // ---- this warp's key range, in 16-key tiles from k_lo
+  // ---- this warp's key range, in kDqKeys-key tiles from k_lo
   const int64_t Nk = a.k.N, Hkv = a.k.H;
   const int64_t s_lo = (int64_t)split * a.keys_per_split;
   const int64_t s_hi = min(Nk, s_lo + a.keys_per_split);
-  const int64_t per_warp = ((s_hi - s_lo + kDqWarps - 1) / kDqWarps + 15) / 16 * 16;
+  const int64_t per_warp = ((s_hi - s_lo + kDqWarps - 1) / kDqWarps + kDqKeys - 1) / kDqKeys * kDqKeys;
   const int64_t k_lo = s_lo + warp * per_warp;
   const int64_t k_hi = min(s_hi, k_lo + per_warp);
   const int64_t qi = a.q_index;
   auto next_visible = [&](int64_t t) {
-    while (t < k_hi && !tile_any_visible(qi, qi, t, min(t + 15, k_hi - 1), a.window, a.n_sink)) {
+    while (t < k_hi && !tile_any_visible(qi, qi, t, min(t + kDqKeys - 1, k_hi - 1), a.window, a.n_sink)) {
       if (t > qi) return k_hi;
-      t += 16;
+      t += kDqKeys;
     }
     return t < k_hi ? t : k_hi;
   };
 
   const int8_t* kbase = reinterpret_cast<const int8_t*>(a.k.ptr) + b * a.k.sb + hk * a.k.sh;
   const int8_t* vbase = reinterpret_cast<const int8_t*>(a.v.ptr) + b * a.v.sb + hk * a.v.sh;
-  const float* ksc = k_scale + b * Nk * Hkv + hk;            // key j: ksc[j * Hkv]
-  const float* vsc = v_scale + b * Nk * Hkv + hk;
+  const float* ksc = k_scale + (b * Hkv + hk) * Nk;          // key j: ksc[j] (head-major scales)
+  const float* vsc = v_scale + (b * Hkv + hk) * Nk;
   uint8_t* wptr = dq_smem + warp * kDqStages * kDqStage;
   const uint32_t wbuf = static_cast<uint32_t>(__cvta_generic_to_shared(wptr));
-  // codes and scales of keys t .. t + 15 -> stage st (keys past the range are zero-filled)
+  // ldmatrix row address of this lane inside a 16-key half of a V tile: matrix
+  // lane / 8 is keys 0-7 or 8-15 (bit 0) and bytes [0, 16) or [16, 32) of a
+  // 32-byte slice (bit 1)
+  const uint32_t v_lane = ((lane & 7) + 8 * ((lane >> 3) & 1)) * kDqRow + 16 * (lane >> 4);
+  // codes and scales of keys t .. t + 31 -> stage st (keys past the range are
+  // zero-filled).  Lane l copies 16-byte piece l % 8 of keys l / 8 + 4i
+  // (i < 8) of both tiles; its global and shared offsets are fixed per lane,
+  // so a tile costs one 64-bit product per operand and constant steps.
+  const int lk = lane >> 3;
+  const int8_t* k_lane = kbase + lk * a.k.sn + (lane & 7) * 16;
+  const int8_t* v_lane_g = vbase + lk * a.v.sn + (lane & 7) * 16;
+  const int64_t k_step = 4 * a.k.sn, v_step = 4 * a.v.sn;
+  const uint32_t s_lane = lk * kDqRow + (lane & 7) * 16;
   auto issue = [&](int64_t t, int st) {
     if (t < k_hi) {
-      const uint32_t ks = wbuf + st * kDqStage;
+      const uint32_t ks = wbuf + st * kDqStage + s_lane;
+      const int8_t* kp = k_lane + t * a.k.sn;
+      const int8_t* vp = v_lane_g + t * a.v.sn;
+      const int64_t rem = k_hi - t;                 // keys of the tile in range (warp-uniform)
+      if (rem >= kDqKeys) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = lane + 32 * i;
-        const int key = e >> 3, col = e & 7;
-        const int64_t j = t + key;
-        const bool ok = j < k_hi;
-        const int64_t jj = ok ? j : t;
-        const int bytes = ok ? 16 : 0;
-        const uint32_t off = key * kDqRow + col * 16;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ks + off),
-                     "l"(kbase + jj * a.k.sn + col * 16), "r"(bytes)
-                     : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ks + kDqTile + off),
-                     "l"(vbase + jj * a.v.sn + col * 16), "r"(bytes)
-                     : "memory");
+        for (int i = 0; i < kDqKeys / 4; ++i) {
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ks + 4 * i * kDqRow), "l"(kp + i * k_step)
+                       : "memory");
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ks + kDqTile + 4 * i * kDqRow),
+                       "l"(vp + i * v_step)
+                       : "memory");
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kDqKeys / 4; ++i) {
+          const bool ok = lk + 4 * i < rem;
+          const int bytes = ok ? 16 : 0;             // zero-fill; the source stays inside the tile's first key
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ks + 4 * i * kDqRow),
+                       "l"(ok ? kp + i * k_step : kp - lk * a.k.sn), "r"(bytes)
+                       : "memory");
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ks + kDqTile + 4 * i * kDqRow),
+                       "l"(ok ? vp + i * v_step : vp - lk * a.v.sn), "r"(bytes)
+                       : "memory");
+        }
       }
       {
-        const int key = lane & 15;
-        const int64_t j = t + key;
-        const bool ok = j < k_hi;
-        const float* src = (lane < 16 ? ksc : vsc) + (ok ? j : t) * Hkv;
-        const uint32_t dst = ks + 2 * kDqTile + (lane < 16 ? 0 : 64) + key * 4;
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(ok ? 4 : 0)
+        const bool ok = lane < rem;
+        const int64_t jj = ok ? t + lane : t;              // one coalesced 128-byte row per operand
+        const uint32_t dst = wbuf + st * kDqStage + 2 * kDqTile + lane * 4;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(ksc + jj), "r"(ok ? 4 : 0)
+                     : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst + 4 * kDqKeys), "l"(vsc + jj),
+                     "r"(ok ? 4 : 0)
                      : "memory");
       }
     }
@@ -360,83 +411,99 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
     for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
 
   int64_t t0 = next_visible(k_lo);
-  int64_t t1 = t0 < k_hi ? next_visible(t0 + 16) : k_hi;
+  int64_t t1 = t0 < k_hi ? next_visible(t0 + kDqKeys) : k_hi;
   issue(t0, 0);
   issue(t1, 1);
   int st = 0;
   while (t0 < k_hi) {
-    const int64_t t2 = t1 < k_hi ? next_visible(t1 + 16) : k_hi;
+    const int64_t t2 = t1 < k_hi ? next_visible(t1 + kDqKeys) : k_hi;
     issue(t2, st == 0 ? 2 : st - 1);
     asm volatile("cp.async.wait_group 2;" ::: "memory");
     __syncwarp();
     const uint8_t* ks = wptr + st * kDqStage;
-    const uint8_t* vs = ks + kDqTile;
     const float* sk = reinterpret_cast<const float*>(ks + 2 * kDqTile);
-    const float* sv_ = sk + 16;
-    // S^T = Kq Q^T: K rows g and g + 8, dims [32c, 32c + 32)
-    uint32_t kw[2][8];
+    const float* sv_ = sk + kDqKeys;
+    // S^T = Kq Q^T for the two 16-key halves u (keys 16u + g, 16u + g + 8 in
+    // this lane's rows), dims [32c, 32c + 32) per lane: two independent chains
+    float sacc[2][4];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const uint4 u0 = *reinterpret_cast<const uint4*>(ks + (g + 8 * r) * kDqRow + 32 * c);
-      const uint4 u1 = *reinterpret_cast<const uint4*>(ks + (g + 8 * r) * kDqRow + 32 * c + 16);
-      kw[r][0] = u0.x; kw[r][1] = u0.y; kw[r][2] = u0.z; kw[r][3] = u0.w;
-      kw[r][4] = u1.x; kw[r][5] = u1.y; kw[r][6] = u1.z; kw[r][7] = u1.w;
+    for (int u = 0; u < 2; ++u) {
+      uint32_t kw[2][8];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint8_t* row = ks + (16 * u + g + 8 * r) * kDqRow + 32 * c;
+        const uint4 u0 = *reinterpret_cast<const uint4*>(row);
+        const uint4 u1 = *reinterpret_cast<const uint4*>(row + 16);
+        kw[r][0] = u0.x; kw[r][1] = u0.y; kw[r][2] = u0.z; kw[r][3] = u0.w;
+        kw[r][4] = u1.x; kw[r][5] = u1.y; kw[r][6] = u1.z; kw[r][7] = u1.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[u][e] = 0.f;
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        const uint32_t fa = kw[0][kc] ^ 0x80808080u, fb = kw[1][kc] ^ 0x80808080u;
+        const uint32_t af[4] = {codes_to_h2_off(fa, 0x4140), codes_to_h2_off(fb, 0x4140),
+                                codes_to_h2_off(fa, 0x4342), codes_to_h2_off(fb, 0x4342)};
+        mma_f16_16816(sacc[u], af, qb[kc][0], qb[kc][1]);
+      }
     }
-    // two accumulator chains (even and odd k chunks) halve the dependent MMA sequence
-    float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sacc2[4] = {0.f, 0.f, 0.f, 0.f};
+    // key scales of this lane's keys (u, r): 16u + g + 8r
+    float skr[2][2], svr[2][2];
 #pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-      const uint32_t fa = kw[0][kc] ^ 0x80808080u, fb = kw[1][kc] ^ 0x80808080u;
-      const uint32_t af[4] = {codes_to_h2_off(fa, 0x4140), codes_to_h2_off(fb, 0x4140), codes_to_h2_off(fa, 0x4342),
-                              codes_to_h2_off(fb, 0x4342)};
-      mma_f16_16816((kc & 1) ? sacc2 : sacc, af, qb[kc][0], qb[kc][1]);
-    }
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
-    // key scales, online softmax per head over keys t0 + g, t0 + g + 8
-    const float ska = sk[g], skb = sk[g + 8];
-    const float sva = sv_[g], svb = sv_[g + 8];
+      for (int r = 0; r < 2; ++r) {
+        skr[u][r] = sk[16 * u + g + 8 * r];
+        svr[u][r] = sv_[16 * u + g + 8 * r];
+      }
     // largest V scale of the tile: scales are >= 0, so their bit patterns order
     // like the values and one integer max-reduction over the warp finds it
-    const float tmax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(sva, svb))));
+    const float lmax = fmaxf(fmaxf(svr[0][0], svr[0][1]), fmaxf(svr[1][0], svr[1][1]));
+    const float tmax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(lmax)));
     const float smax_new = fmaxf(smax, tmax);
     const float ratio = smax_new > 0.f ? smax / smax_new : 1.f;
     const float inv_smax = smax_new > 0.f ? 1.f / smax_new : 0.f;
     smax = smax_new;
-    const int64_t ja = t0 + g, jb = t0 + g + 8;
-    const bool va = ja < k_hi && mask_visible(qi, ja, a.window, a.n_sink);
-    const bool vb = jb < k_hi && mask_visible(qi, jb, a.window, a.n_sink);
-    float sv[4];
-    sv[0] = va ? (sacc[0] - qs[0]) * ska * a.scale_log2 : -INFINITY;
-    sv[1] = va ? (sacc[1] - qs[1]) * ska * a.scale_log2 : -INFINITY;
-    sv[2] = vb ? (sacc[2] - qs[0]) * skb * a.scale_log2 : -INFINITY;
-    sv[3] = vb ? (sacc[3] - qs[1]) * skb * a.scale_log2 : -INFINITY;
-    float p[4], beta[2];
+    // per-key mask only on tiles that are ragged or cut by the mask (warp-uniform)
+    bool vis[2][2] = {{true, true}, {true, true}};
+    if (t0 + kDqKeys > k_hi || !tile_all_visible(qi, qi, t0, t0 + kDqKeys - 1, a.window, a.n_sink)) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int64_t j = t0 + 16 * u + g + 8 * r;
+          vis[u][r] = j < k_hi && mask_visible(qi, j, a.window, a.n_sink);
+        }
+    }
+    // logits in log2 units: fragment element e of half u is (key 16u + g + 8(e >> 1), head 2c + (e & 1))
+    float sv[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = e >> 1;
+        sv[u][e] = vis[u][r] ? (sacc[u][e] - qs[e & 1]) * skr[u][r] * a.scale_log2 : -INFINITY;
+      }
+    float p[2][4], beta[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float mx = fmaxf(sv[h], sv[h + 2]);
+      float mx = fmaxf(fmaxf(sv[0][h], sv[0][h + 2]), fmaxf(sv[1][h], sv[1][h + 2]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float m_new = fmaxf(m[h], mx);
       const float mref = m_new == -INFINITY ? 0.f : m_new;
       const float alpha = dec_exp2(m[h] - mref);
-      p[h] = dec_exp2(sv[h] - mref);
-      p[h + 2] = dec_exp2(sv[h + 2] - mref);
-      l[h] = l[h] * alpha + (p[h] + p[h + 2]);
+      float sum = 0.f;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        p[u][h] = dec_exp2(sv[u][h] - mref);
+        p[u][h + 2] = dec_exp2(sv[u][h + 2] - mref);
+        sum += p[u][h] + p[u][h + 2];
+      }
+      l[h] = l[h] * alpha + sum;
       m[h] = m_new;
       beta[h] = alpha * ratio;
-    }
-    // P' = p * s_v / s_max, transposed into the B operand of the P V product
-    const float wa = sva * inv_smax, wb = svb * inv_smax;
-    const uint32_t pb0 = movmatrix_t(f2_to_h2(p[0] * wa, p[1] * wa));   // keys 2c, 2c + 1 of head g
-    const uint32_t pb1 = movmatrix_t(f2_to_h2(p[2] * wb, p[3] * wb));   // keys 2c + 8, 2c + 9
-    // O^T = beta O^T + Vq^T P'^T: V rows 2c, 2c + 1, 2c + 8, 2c + 9, dims [16g, 16g + 16)
-    uint4 vr[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int key = 2 * c + (i & 1) + 8 * (i >> 1);
-      vr[i] = *reinterpret_cast<const uint4*>(vs + key * kDqRow + 16 * g);
     }
     // O rescale only when some column's factor moved (the max or s_max grew)
     if (__any_sync(0xffffffffu, beta[0] != 1.f || beta[1] != 1.f)) {
@@ -448,17 +515,29 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
         o[mt][3] *= beta[1];
       }
     }
+    // O^T += Vq^T P'^T per half u, P' = p * s_v / s_max transposed into the B
+    // operand.  ldmatrix.trans of the V codes (16-bit elements = two dims of
+    // one key) gives lane (g, c) dims 2g, 2g + 1 of keys 2c, 2c + 1 in one
+    // register, so two byte selections make A rows "dim 16 mt + 2g" (row g)
+    // and "dim 16 mt + 2g + 1" (row g + 8).
+    const uint32_t vs_lane = wbuf + st * kDqStage + kDqTile + v_lane;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      // operand rows: dim 16g + 2mt (row g) and 16g + 2mt + 1 (row g + 8)
-      const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;   // bytes j, j + 1 of two keys, interleaved
-      const int wi = mt >> 1;
-      auto word = [](const uint4& u, int i) { return i == 0 ? u.x : i == 1 ? u.y : i == 2 ? u.z : u.w; };
-      const uint32_t lo = __byte_perm(word(vr[0], wi), word(vr[1], wi), sel) ^ 0x80808080u;   // keys 2c, 2c+1
-      const uint32_t hi = __byte_perm(word(vr[2], wi), word(vr[3], wi), sel) ^ 0x80808080u;   // keys 2c+8, 2c+9
-      const uint32_t af[4] = {codes_to_h2(lo, 0x4140), codes_to_h2(lo, 0x4342), codes_to_h2(hi, 0x4140),
-                              codes_to_h2(hi, 0x4342)};
-      mma_f16_16816(o[mt], af, pb0, pb1);
+    for (int u = 0; u < 2; ++u) {
+      const float wa = svr[u][0] * inv_smax, wb = svr[u][1] * inv_smax;
+      const uint32_t pb0 = movmatrix_t(f2_to_h2(p[u][0] * wa, p[u][1] * wa));   // keys 2c, 2c + 1 of head g
+      const uint32_t pb1 = movmatrix_t(f2_to_h2(p[u][2] * wb, p[u][3] * wb));   // keys 2c + 8, 2c + 9
+#pragma unroll
+      for (int mp = 0; mp < 4; ++mp) {
+        uint32_t rr[4];
+        ldsm_x4_t(rr, vs_lane + 16 * u * kDqRow + 32 * mp);   // rr0/rr1: keys 0-7 / 8-15, dims 32mp + [0, 16); rr2/rr3: + 16
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t x0 = rr[2 * h] ^ 0x80808080u, x1 = rr[2 * h + 1] ^ 0x80808080u;
+          const uint32_t af[4] = {codes_to_h2(x0, 0x4240), codes_to_h2(x0, 0x4341), codes_to_h2(x1, 0x4240),
+                                  codes_to_h2(x1, 0x4341)};
+          mma_f16_16816(o[2 * mp + h], af, pb0, pb1);
+        }
+      }
     }
     __syncwarp();   // stage st is refilled two iterations on
     st = st == kDqStages - 1 ? 0 : st + 1;
@@ -484,8 +563,8 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
   }
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
-    // C rows: g -> dim 16g + 2mt, g + 8 -> dim 16g + 2mt + 1; columns: heads 2c, 2c + 1
-    float* w0 = sm_o + (warp * kDecMaxG + 2 * c) * 128 + 16 * g + 2 * mt;
+    // C rows: g -> dim 16mt + 2g, g + 8 -> dim 16mt + 2g + 1; columns: heads 2c, 2c + 1
+    float* w0 = sm_o + (warp * kDecMaxG + 2 * c) * 128 + 16 * mt + 2 * g;
     w0[0] = o[mt][0] * smax;
     w0[128] = o[mt][1] * smax;
     w0[1] = o[mt][2] * smax;

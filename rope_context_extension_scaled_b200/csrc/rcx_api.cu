@@ -452,11 +452,11 @@ int quantize_i8_impl(const rcx_tensor& x, const rcx_tensor& c, float* scale, cud
   a.c = make_view(c);
   a.scale = scale;
   a.rows = rows;
-  auto packed = [](const rcx_tensor& t) {     // [B, N, H, 128] with no gaps
-    return t.stride[3] == 1 && t.stride[2] == 128 && t.stride[1] == t.shape[2] * 128 &&
-           (t.shape[0] == 1 || t.stride[0] == t.shape[1] * t.stride[1]);
-  };
-  a.dense = packed(x) && packed(c);
+  a.fast = rows < (int64_t(1) << 31);
+  if (a.fast) {
+    a.div_h = make_fastdiv((uint32_t)x.shape[2]);
+    a.div_n = make_fastdiv((uint32_t)x.shape[1]);
+  }
   const bool rows16 = aligned_rows(x, 16) && aligned_rows(c, 16);
   const int64_t per_cta = rows16 ? 32 : 8;      // rows a CTA covers per pass (four or one per warp)
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((rows + per_cta - 1) / per_cta,

@@ -51,7 +51,7 @@ def test_quantize_codes_and_scales_bit_exact(B, Nk, Hkv):
     torch.cuda.synchronize()
     c_ref, s_ref = orc.quantize_kv_int8(x.float().cpu().numpy())
     assert np.array_equal(codes.cpu().numpy(), c_ref)
-    assert np.array_equal(scale.cpu().numpy(), s_ref)
+    assert np.array_equal(scale.permute(0, 2, 1).cpu().numpy(), s_ref)   # device scales are [B, H, N]
 
 
 def test_quantize_strided_view():
@@ -64,7 +64,7 @@ def test_quantize_strided_view():
     torch.cuda.synchronize()
     c_ref, s_ref = orc.quantize_kv_int8(base.float().cpu().numpy())
     assert np.array_equal(codes.cpu().numpy(), c_ref)
-    assert np.array_equal(scale.cpu().numpy(), s_ref)
+    assert np.array_equal(scale.permute(0, 2, 1).cpu().numpy(), s_ref)   # device scales are [B, H, N]
     assert not out[:, :, 4].any()                          # nothing written outside the view
 
 
@@ -81,7 +81,7 @@ def test_quantize_8_byte_rows_and_odd_row_count():
         torch.cuda.synchronize()
         c_ref, s_ref = orc.quantize_kv_int8(base.float().cpu().numpy())
         assert np.array_equal(codes.cpu().numpy(), c_ref)
-        assert np.array_equal(scale.cpu().numpy(), s_ref)
+        assert np.array_equal(scale.permute(0, 2, 1).cpu().numpy(), s_ref)   # device scales are [B, H, N]
 
 
 def _oracle_decode(q, k, v, inv_freq, t, q_index, window, n_sink):
