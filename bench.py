@@ -36,10 +36,14 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "causal attention fwd TFLOP/s and % of B200 BF16 tensor peak at 128K and 1M"
-# DRAM bytes (read + write) per attention launch of the named workload, from an
-# ncu capture of the attention kernel as currently built (empty until one is
-# taken; reported as roofline.traffic).
-ATTN_TRAFFIC_PER_LAUNCH = {}
+# DRAM bytes (read + write) per attention launch of the named workload from
+# ncu captures of the attention kernel as currently built, reported as
+# roofline.traffic (remove an entry when the kernel changes).  32K: one launch
+# captured.  1M: not captured at full size; the four launch forms of its ring
+# were captured on the three-block 192K ring (same heads, block size and
+# schedule) and weighted by their counts in the 1M step (1 direct, 15 first,
+# 105 middle, 15 last).
+ATTN_TRAFFIC_PER_LAUNCH = {"llama3_70b_32k_yarn": 1.193e9, "llama3_70b_1m_ring": 5.676e9}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
