@@ -464,12 +464,17 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a)
     const int64_t row = e / 32;
     const int c = (int)(e % 32);
     const int64_t b = row / a.q.H, h = row % a.q.H;
+    // max of the partial LSEs: lane c reads splits c, c + 32, ... and the row's
+    // 32 lanes (one warp) reduce, so the reads of all splits are in flight at once
     float mm = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) mm = fmaxf(mm, a.part_lse[(int64_t)s * rows + row]);
+    for (int s = c; s < a.splits; s += 32) mm = fmaxf(mm, a.part_lse[(int64_t)s * rows + row]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
     float lse = -INFINITY;
     if (mm != -INFINITY) {
       float wsum = 0.f;
+#pragma unroll 8
       for (int s = 0; s < a.splits; ++s) {
         const float ls = a.part_lse[(int64_t)s * rows + row];
         const float w = ls == -INFINITY ? 0.f : expf(ls - mm);

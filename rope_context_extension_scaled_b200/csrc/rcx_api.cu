@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <mutex>
 #include <vector>
 
@@ -560,10 +561,20 @@ RingPlan ring_plan(const rcx_tensor& q, const rcx_tensor& k, int64_t kv_block, i
   return p;
 }
 
+// Points where a caller that streams the inputs in and the outputs out (the
+// host-buffer entry point) joins the ring schedule on its stream: before the
+// first kernel that reads K, before the launch of query shard r against key
+// block b, and after the launch that writes shard r's final output.
+struct RingHooks {
+  std::function<int()> before_k;
+  std::function<int(int64_t r, int64_t b)> before_launch;
+  std::function<int(int64_t r)> after_final;
+};
+
 int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, const rcx_tensor& o,
               const rcx_tensor& lse, int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
               const int64_t* positions, int64_t n_positions, const double* inv_freq, int rope_flags,
-              void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
+              void* workspace, int64_t workspace_bytes, cudaStream_t stream, const RingHooks* hooks = nullptr) {
   int st;
   if ((st = check_act(q)) || (st = check_act(k)) || (st = check_act(v)) || (st = check_act(o))) return st;
   if (k.shape[1] != q.shape[1]) return RCX_ERR_INVALID_ARG;     // self-attention over one sequence
@@ -578,6 +589,7 @@ int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
 
   rcx_tensor kk = k;
   int flags = rope_flags;
+  if (hooks && (st = hooks->before_k())) return st;
   if (p.rotate_k_separately) {
     // K is shared by G query heads and by every query tile: rotate it once.
     rcx_tensor krot = make_tensor(ws + p.off_krot, RCX_BF16, p.B, p.N, p.Hkv, p.D);
@@ -611,10 +623,12 @@ int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
       rcx_tensor vs = token_slice(v, j0, nj);
       rcx_tensor os_final = token_slice(o, i0, ni);
       rcx_tensor ls_final = lse.ptr ? lse_slice(lse, i0, ni) : null_tensor();
+      if (hooks && (st = hooks->before_launch(r, b))) return st;
       if (count[r] == 1) {          // one visible block: write the result directly
         st = attn_impl(qs, ks, vs, os_final, ls_final, 0, window, n_sink, temperature, i0, j0, positions,
                        n_positions, inv_freq, flags, stream);
         if (st) return st;
+        if (hooks && (st = hooks->after_final(r))) return st;
         continue;
       }
       rcx_tensor as = token_slice(acc, i0, ni);
@@ -631,12 +645,35 @@ int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
                        inv_freq, flags, stream, &as, &las);
       }
       if (st) return st;
+      if (hooks && t == last[r] && (st = hooks->after_final(r))) return st;
     }
   }
   return RCX_OK;
 }
 
 }  // namespace
+
+// Copy streams and events of rcx_ring_attn_fwd_host; released by the
+// destructor (after the call has synchronised them).
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  std::vector<cudaEvent_t> events;
+  bool ok = true;
+  cudaEvent_t event() {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      ok = false;
+      return nullptr;
+    }
+    events.push_back(e);
+    return e;
+  }
+  ~HostPipe() {
+    for (cudaEvent_t e : events) cudaEventDestroy(e);
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+};
 
 // =============================================================== C entry points
 
@@ -750,6 +787,8 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
         t.stride[0] != t.shape[1] * t.stride[1])
       return RCX_ERR_INVALID_ARG;
   }
+  if (k.shape[1] != q.shape[1] || v.shape[1] != q.shape[1] || o.shape[1] != q.shape[1] || kv_block < 0)
+    return RCX_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   auto bytes = [](const rcx_tensor& t) {
     return t.shape[0] * t.shape[1] * t.shape[2] * t.shape[3] * (int64_t)elem_size(t.dtype);
@@ -761,33 +800,103 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
   const int64_t sizes[7] = {bytes(q), bytes(k), bytes(v), bytes(o), lse_bytes, ws_bytes, pos_bytes};
   int64_t offs[7], total = 0;
   for (int i = 0; i < 7; ++i) { offs[i] = total; total = align256(total + sizes[i]); }
+  const RingPlan plan = ring_plan(q, k, kv_block, rope_flags);
+  const int64_t P = std::max<int64_t>(plan.P, 1);
+
+  // The copies run on two streams of their own and meet the schedule on `s`
+  // through events: K and the positions first (the K rotation reads all of
+  // K), then shard r's query rows with block r's V rows in ring order, so the
+  // launches of shard r wait only for what they read; each shard's final
+  // output goes back as soon as its last launch is done.
+  HostPipe hp;
   char* dev = nullptr;
+  int st = RCX_OK;
+  auto ck = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == RCX_OK) st = RCX_ERR_CUDA;
+    return st == RCX_OK;
+  };
+  if (!ck(cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking)) ||
+      !ck(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)))
+    return st;
   if (cudaMallocAsync(reinterpret_cast<void**>(&dev), (size_t)std::max<int64_t>(total, 256), s) != cudaSuccess)
     return RCX_ERR_CUDA;
   rcx_tensor dq = q, dk = k, dv = v, dout = o, dl = lse;
   dq.ptr = dev + offs[0]; dk.ptr = dev + offs[1]; dv.ptr = dev + offs[2]; dout.ptr = dev + offs[3];
   if (lse.ptr) dl.ptr = dev + offs[4];
   int64_t* dpos = positions ? reinterpret_cast<int64_t*>(dev + offs[6]) : nullptr;
-  int st = RCX_OK;
-  if (cudaMemcpyAsync(dq.ptr, q.ptr, sizes[0], cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk.ptr, k.ptr, sizes[1], cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv.ptr, v.ptr, sizes[2], cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      (dpos && cudaMemcpyAsync(dpos, positions, pos_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess))
-    st = RCX_ERR_CUDA;
-  if (!st)
+
+  // rows [r kv, min((r + 1) kv, N)) of every batch entry of a dense [B, N, H, d] tensor
+  auto copy_rows = [&](void* dst, const void* src, const rcx_tensor& t, int64_t r, cudaMemcpyKind kind,
+                       cudaStream_t cs) {
+    const int64_t row_bytes = t.shape[2] * t.shape[3] * elem_size(t.dtype);
+    const int64_t i0 = r * plan.kv, ni = std::min((r + 1) * plan.kv, t.shape[1]) - i0;
+    for (int64_t b = 0; b < t.shape[0] && st == RCX_OK && ni > 0; ++b) {
+      const int64_t off = (b * t.shape[1] + i0) * row_bytes;
+      ck(cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, ni * row_bytes, kind,
+                         cs));
+    }
+  };
+  cudaEvent_t ev_alloc = hp.event(), ev_k = hp.event();
+  std::vector<cudaEvent_t> ev_in(P);
+  for (int64_t r = 0; r < P; ++r) ev_in[r] = hp.event();
+  if (!hp.ok) st = RCX_ERR_CUDA;
+  if (ck(cudaEventRecord(ev_alloc, s)) && ck(cudaStreamWaitEvent(hp.in, ev_alloc, 0)) &&
+      ck(cudaStreamWaitEvent(hp.out, ev_alloc, 0)) &&
+      ck(cudaMemcpyAsync(dk.ptr, k.ptr, sizes[1], cudaMemcpyHostToDevice, hp.in)) &&
+      (!dpos || ck(cudaMemcpyAsync(dpos, positions, pos_bytes, cudaMemcpyHostToDevice, hp.in))) &&
+      ck(cudaEventRecord(ev_k, hp.in))) {
+    for (int64_t r = 0; r < P && st == RCX_OK; ++r) {
+      copy_rows(dq.ptr, q.ptr, q, r, cudaMemcpyHostToDevice, hp.in);
+      copy_rows(dv.ptr, v.ptr, v, r, cudaMemcpyHostToDevice, hp.in);
+      ck(cudaEventRecord(ev_in[r], hp.in));
+    }
+  }
+
+  std::vector<char> handed(P, 0);
+  int64_t waited = -1;
+  RingHooks hooks;
+  hooks.before_k = [&]() -> int {
+    return cudaStreamWaitEvent(s, ev_k, 0) == cudaSuccess ? RCX_OK : RCX_ERR_CUDA;
+  };
+  hooks.before_launch = [&](int64_t r, int64_t b) -> int {
+    const int64_t m = std::max(r, b);
+    if (m > waited) {
+      if (cudaStreamWaitEvent(s, ev_in[m], 0) != cudaSuccess) return RCX_ERR_CUDA;
+      waited = m;
+    }
+    return RCX_OK;
+  };
+  hooks.after_final = [&](int64_t r) -> int {
+    cudaEvent_t e = hp.event();
+    if (!e || cudaEventRecord(e, s) != cudaSuccess || cudaStreamWaitEvent(hp.out, e, 0) != cudaSuccess)
+      return RCX_ERR_CUDA;
+    copy_rows(o.ptr, dout.ptr, o, r, cudaMemcpyDeviceToHost, hp.out);
+    handed[r] = 1;
+    return st;
+  };
+  if (st == RCX_OK)
     st = ring_impl(dq, dk, dv, dout, dl, kv_block, window, n_sink, temperature, dpos, n_positions, inv_freq,
-                   rope_flags, dev + offs[5], ws_bytes, s);
-  if (!st && (cudaMemcpyAsync(o.ptr, dout.ptr, sizes[3], cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-              (lse.ptr && cudaMemcpyAsync(lse.ptr, dl.ptr, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)))
-    st = RCX_ERR_CUDA;
+                   rope_flags, dev + offs[5], ws_bytes, s, &hooks);
+  // after the schedule: the LSE and any output not handed out yet
+  if (st == RCX_OK) {
+    cudaEvent_t e_end = hp.event();
+    if (ck(e_end ? cudaEventRecord(e_end, s) : cudaErrorUnknown) && ck(cudaStreamWaitEvent(hp.out, e_end, 0))) {
+      for (int64_t r = 0; r < P && st == RCX_OK; ++r)
+        if (!handed[r]) copy_rows(o.ptr, dout.ptr, o, r, cudaMemcpyDeviceToHost, hp.out);
+      if (lse.ptr) ck(cudaMemcpyAsync(lse.ptr, dl.ptr, lse_bytes, cudaMemcpyDeviceToHost, hp.out));
+    }
+  }
+  // Both copy streams finish before the device memory is released (on every path).
+  if (cudaStreamSynchronize(hp.in) != cudaSuccess && st == RCX_OK) st = RCX_ERR_CUDA;
+  if (cudaStreamSynchronize(hp.out) != cudaSuccess && st == RCX_OK) st = RCX_ERR_CUDA;
   cudaFreeAsync(dev, s);
-  if (cudaStreamSynchronize(s) != cudaSuccess && !st) st = RCX_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess && st == RCX_OK) st = RCX_ERR_CUDA;
   // This call is synchronous, so a bounded wait that ran out in one of its
   // kernels is reported here (and the status word cleared), not left for a
   // later rcx_device_status().
   int dev_st = RCX_OK;
-  if (!st && device_status_all(s, &dev_st) != RCX_OK) st = RCX_ERR_CUDA;
-  if (!st && dev_st != RCX_OK) st = dev_st;
+  if (st == RCX_OK && device_status_all(s, &dev_st) != RCX_OK) st = RCX_ERR_CUDA;
+  if (st == RCX_OK && dev_st != RCX_OK) st = dev_st;
   return st;
 }
 

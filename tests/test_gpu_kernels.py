@@ -372,6 +372,35 @@ def test_ring_host_buffers_entry_point():
     assert torch.equal(oh, od.cpu()) and torch.equal(lh, ld.cpu())
 
 
+@pytest.mark.parametrize("B,N,Hq,Hkv,d,dtype,kv,window,n_sink,use_pos", [
+    (2, 700, 4, 2, 128, torch.bfloat16, 128, 100, 3, True),     # ragged last block, batch 2, mask, positions
+    (1, 300, 2, 1, 64, torch.float32, 64, 0, 0, False),         # fp32 path: K rotated in the kernel
+    (1, 256, 4, 1, 128, torch.bfloat16, 0, 0, 0, False),        # one block
+])
+def test_ring_host_pipeline_matches_device_path(B, N, Hq, Hkv, d, dtype, kv, window, n_sink, use_pos):
+    # The host entry point streams shard r's Q and V rows in, and shard r's
+    # output out, on copy streams joined to the schedule by events: the result
+    # must be the device-buffer result, bit for bit.
+    q, k, v = make_qkv(B, N, Hq, Hkv, d, dtype, seed=17, device="cpu")
+    inv, t, _, _ = schedule(_lib.YARN, 1e4, d, 128, 1024)
+    pos = None
+    if use_pos:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(5)
+        pos = torch.randint(0, 1 << 20, (N,), generator=g, dtype=torch.int64)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(B, Hq, N, dtype=torch.float32).pin_memory()
+    flags = _lib.ROTATE_Q | _lib.ROTATE_K
+    _lib.ring_attn_fwd_host(qh, kh, vh, oh, lh, kv_block=kv, window=window, n_sink=n_sink, temperature=t,
+                            positions=pos, inv_freq=inv, rope_flags=flags)
+    od, ld = _lib.ring_attn_fwd(q.cuda(), k.cuda(), v.cuda(), kv_block=kv, window=window, n_sink=n_sink,
+                                temperature=t, positions=None if pos is None else pos.cuda(), inv_freq=inv,
+                                rope_flags=flags)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, od.cpu()) and torch.equal(lh, ld.cpu())
+
+
 # ------------------------------------------------------------ bounded waits
 
 def test_bounded_wait_timeout_reports_and_context_survives():
