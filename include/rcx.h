@@ -330,17 +330,31 @@ int rcx_ring_attn_fwd_noalloc(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tens
 /*
  * Host<->device convenience for callers without device memory management:
  * same as rcx_ring_attn_fwd but q, k, v, o (and lse if non-NULL) are HOST
- * buffers (pinned for full copy speed); the call allocates the device copies
- * and workspace, copies in, computes, copies out and frees, synchronously on
- * `stream`.  positions is a HOST array here.  Because the call synchronises,
- * it also reads (and clears) the device status words: a bounded wait that ran
- * out in one of its kernels returns RCX_ERR_DEVICE_TIMEOUT (o and lse then
- * hold incomplete results).
+ * buffers (pinned for full copy speed; dense [B, N, H, d] and [B, H, N, 1]);
+ * the call stages device copies and the workspace, streams the inputs in
+ * (K first, then each query shard with its V block) and each shard's output
+ * out as soon as it is final, on two copy streams of its own joined to
+ * `stream` by events, and returns when everything is back on the host.
+ * positions is a HOST array here.  The staging memory comes from a
+ * library-owned memory pool of the current device that keeps it after the
+ * call, so that repeated calls do not map it again (mapping ~73 GB costs
+ * about a second on B200); rcx_release_staging() hands it back.  Because the
+ * call synchronises, it also reads (and clears) the device status words: a
+ * bounded wait that ran out in one of its kernels returns
+ * RCX_ERR_DEVICE_TIMEOUT (o and lse then hold incomplete results).
  */
 int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor o, rcx_tensor lse,
                            int64_t kv_block, int64_t window, int64_t n_sink, double temperature,
                            const int64_t* positions, int64_t n_positions, const double* inv_freq,
                            int rope_flags, void* stream);
+
+/*
+ * Returns the device memory that rcx_ring_attn_fwd_host keeps between calls
+ * (every device's pool is trimmed to zero; memory of a call still running is
+ * not touched).  Safe to call at any time; RCX_ERR_CUDA if the runtime
+ * refuses.
+ */
+int rcx_release_staging(void);
 
 /*
  * Device status word: kernels with bounded waits record the first

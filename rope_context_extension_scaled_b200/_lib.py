@@ -32,7 +32,7 @@ EXPORTS = (
     "rcx_debug_inject_wait_timeout", "rcx_stats_enable_timing", "rcx_stats_reset", "rcx_stats_read",
     "rcx_ring_attn_fwd_noalloc", "rcx_rope_freqs_per_pair", "rcx_attn_decode_workspace_size",
     "rcx_attn_decode_fwd", "rcx_kv_quantize_int8", "rcx_attn_decode_int8_workspace_size",
-    "rcx_attn_decode_int8_fwd", "rcx_attn_blockwise_merge_fwd",
+    "rcx_attn_decode_int8_fwd", "rcx_attn_blockwise_merge_fwd", "rcx_release_staging",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20   # RCX_NOALLOC_SCRATCH_BYTES in include/rcx.h
 KERNEL_KINDS = {"rope_apply": 0, "attn_tc": 1, "attn_simt": 2, "merge": 3, "decode": 4}
@@ -85,6 +85,8 @@ def load():
     lib.rcx_attn_blockwise_merge_fwd.argtypes = [T, T, T, T, T, T, T, i64, i64, i64, f64, i64, i64, vp, i64, pd,
                                                  ctypes.c_int, vp]
     lib.rcx_attn_blockwise_merge_fwd.restype = ctypes.c_int
+    lib.rcx_release_staging.argtypes = []
+    lib.rcx_release_staging.restype = ctypes.c_int
     lib.rcx_merge_partials.argtypes = [T, T, T, T, T, T, vp]
     lib.rcx_ring_workspace_size.argtypes = [T, T, i64, ctypes.c_int]
     lib.rcx_ring_workspace_size.restype = i64
@@ -285,6 +287,11 @@ def ring_attn_fwd_host(q, k, v, o, lse=None, kv_block=0, window=0, n_sink=0, tem
                                        int(window), int(n_sink), float(temperature), pp, npos, fp, int(rope_flags), s)
     _check(st, "rcx_ring_attn_fwd_host")
     return o, lse
+
+
+def release_staging():
+    """Return the staging memory rcx_ring_attn_fwd_host keeps between calls."""
+    _check(load().rcx_release_staging(), "rcx_release_staging")
 
 
 def device_status(device=None):

@@ -653,6 +653,55 @@ int ring_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, con
 
 }  // namespace
 
+namespace {
+
+// Staging memory of rcx_ring_attn_fwd_host: one pool per device that keeps
+// what it has mapped (release threshold: all), so that a repeated call reuses
+// the ~73 GB of a 1M-token call instead of mapping it again; handed back by
+// rcx_release_staging.
+constexpr int kMaxDevices = 64;
+std::mutex g_staging_mu;
+cudaMemPool_t g_staging[kMaxDevices] = {};
+
+cudaError_t staging_pool(int dev, bool fresh, cudaMemPool_t* out) {
+  std::lock_guard<std::mutex> lock(g_staging_mu);
+  if (fresh) g_staging[dev] = nullptr;          // a handle that stopped working (context re-created)
+  if (!g_staging[dev]) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = UINT64_MAX;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    g_staging[dev] = pool;
+  }
+  *out = g_staging[dev];
+  return cudaSuccess;
+}
+
+cudaError_t staging_alloc(void** p, size_t bytes, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaMallocAsync(p, bytes, s);
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    cudaMemPool_t pool = nullptr;
+    if ((e = staging_pool(dev, attempt > 0, &pool)) != cudaSuccess) return e;
+    if ((e = cudaMallocFromPoolAsync(p, bytes, pool, s)) == cudaSuccess) return e;
+    if (e == cudaErrorMemoryAllocation) return e;
+    cudaGetLastError();                         // clear, and retry once with a new pool
+  }
+  return e;
+}
+
 // Copy streams and events of rcx_ring_attn_fwd_host; released by the
 // destructor (after the call has synchronised them).
 struct HostPipe {
@@ -674,6 +723,8 @@ struct HostPipe {
     if (out) cudaStreamDestroy(out);
   }
 };
+
+}  // namespace
 
 // =============================================================== C entry points
 
@@ -818,7 +869,7 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
   if (!ck(cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking)) ||
       !ck(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking)))
     return st;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&dev), (size_t)std::max<int64_t>(total, 256), s) != cudaSuccess)
+  if (staging_alloc(reinterpret_cast<void**>(&dev), (size_t)std::max<int64_t>(total, 256), s) != cudaSuccess)
     return RCX_ERR_CUDA;
   rcx_tensor dq = q, dk = k, dv = v, dout = o, dl = lse;
   dq.ptr = dev + offs[0]; dk.ptr = dev + offs[1]; dv.ptr = dev + offs[2]; dout.ptr = dev + offs[3];
@@ -897,6 +948,14 @@ int rcx_ring_attn_fwd_host(rcx_tensor q, rcx_tensor k, rcx_tensor v, rcx_tensor 
   int dev_st = RCX_OK;
   if (st == RCX_OK && device_status_all(s, &dev_st) != RCX_OK) st = RCX_ERR_CUDA;
   if (st == RCX_OK && dev_st != RCX_OK) st = dev_st;
+  return st;
+}
+
+int rcx_release_staging(void) {
+  std::lock_guard<std::mutex> lock(g_staging_mu);
+  int st = RCX_OK;
+  for (int d = 0; d < kMaxDevices; ++d)
+    if (g_staging[d] && cudaMemPoolTrimTo(g_staging[d], 0) != cudaSuccess) st = RCX_ERR_CUDA;
   return st;
 }
 

@@ -32,6 +32,11 @@ def test_library_exports_every_declared_symbol(lib):
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
 
 
+def test_release_staging_without_pools_is_a_no_op(lib):
+    # no host-buffer call has run in this process: nothing to trim, no CUDA call
+    assert lib.rcx_release_staging() == 0
+
+
 def test_version_and_status_strings(lib):
     assert lib.rcx_abi_version() == 100
     assert _lib.status_string(0) == "ok"

@@ -401,6 +401,30 @@ def test_ring_host_pipeline_matches_device_path(B, N, Hq, Hkv, d, dtype, kv, win
     assert torch.equal(oh, od.cpu()) and torch.equal(lh, ld.cpu())
 
 
+def test_ring_host_staging_kept_and_released():
+    # The host entry point keeps its staging memory in a library pool between
+    # calls; repeated calls, a release, and a call after it give one result.
+    N = 384
+    q, k, v = make_qkv(1, N, 4, 2, 128, torch.bfloat16, seed=18, device="cpu")
+    inv, t, _, _ = schedule(_lib.NTK, 5e5, 128, 256, 1024)
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    outs = []
+    for release in (False, False, True):
+        oh = torch.empty_like(qh).pin_memory()
+        lh = torch.empty(1, 4, N, dtype=torch.float32).pin_memory()
+        _lib.ring_attn_fwd_host(qh, kh, vh, oh, lh, kv_block=128, temperature=t, inv_freq=inv,
+                                rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+        outs.append((oh, lh))
+        if release:
+            _lib.release_staging()
+    oh, lh = torch.empty_like(qh).pin_memory(), torch.empty(1, 4, N, dtype=torch.float32).pin_memory()
+    _lib.ring_attn_fwd_host(qh, kh, vh, oh, lh, kv_block=128, temperature=t, inv_freq=inv,
+                            rope_flags=_lib.ROTATE_Q | _lib.ROTATE_K)
+    outs.append((oh, lh))
+    for o_, l_ in outs[1:]:
+        assert torch.equal(o_, outs[0][0]) and torch.equal(l_, outs[0][1])
+
+
 # ------------------------------------------------------------ bounded waits
 
 def test_bounded_wait_timeout_reports_and_context_survives():
