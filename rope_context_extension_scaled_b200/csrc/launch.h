@@ -66,7 +66,7 @@ int decode_launch(const DecodeArgs& a, int G, bool tensor_core, dim3 grid, cudaS
 int decode_i8_launch(const DecodeArgs& a, int G, const float* k_scale, const float* v_scale, dim3 grid,
                      cudaStream_t stream);
 int decode_combine_launch(const DecodeArgs& a, int out_dtype, int grid, cudaStream_t stream);
-// rows16: bf16 rows 16-byte and code rows 8-byte aligned (half-warp-per-row kernel)
+// rows16: bf16 rows and code rows both 16-byte aligned (eight-lanes-per-row kernel)
 int quantize_i8_launch(const QuantArgs& a, bool rows16, int grid, cudaStream_t stream);
 
 // Device status words: every translation unit whose kernels have bounded
