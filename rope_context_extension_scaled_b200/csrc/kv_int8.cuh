@@ -14,17 +14,19 @@
 // columns), with 32-key tiles so that a tile moves as many bytes as the bf16
 // kernel's 16-key tile and the per-tile softmax work is shared by 32 keys, and
 // the dequantisation in the tile load:
-//  * the MMAs run in fp16 (m16n8k16, fp32 accumulate), because an int8 code
-//    becomes an exact fp16 in three integer/half instructions: the byte with
-//    its sign bit flipped (u = code + 128) is placed under the exponent
-//    pattern of 1024, which reads as 1024 + u, and 1152 is subtracted;
-//  * K codes go into S^T = Kq Q^T unscaled and without the subtraction, i.e.
-//    as code + 1152 (two instructions per pair of codes): the product then
-//    carries 1152 sum_d q_d per query head, which is removed from S^T in fp32
-//    (the products are exact in fp32 and |S'| stays near 1e4, so the
-//    cancellation costs about 1e-5 of the logit); each key's scale then
-//    multiplies its row of S^T.  The V path keeps the subtraction: there the
-//    offset would grow with the number of keys summed into O;
+//  * S^T = Kq Q^T runs on int8 MMAs (m16n8k32, int32 accumulate) with the
+//    codes as they are stored: the rotated query of each head is split as
+//    q = s_q (128 hi + lo) + e, hi in [-127, 127], lo in [-64, 64],
+//    |e| <= s_q / 2 with s_q = amax / (127 * 128), and two MMAs per 32 dims
+//    give codes . hi and codes . lo exactly; 128 hi-part + lo-part (|.| < 2^29)
+//    times s_q and the key's scale is the logit.  The query error is 15 bits
+//    of its largest element, finer than an fp16 operand;
+//  * the P V product runs in fp16 (m16n8k16, fp32 accumulate), because an int8
+//    code becomes an exact fp16 in three integer/half instructions: the byte
+//    with its sign bit flipped (u = code + 128) is placed under the exponent
+//    pattern of 1024, which reads as 1024 + u, and 1152 is subtracted (the
+//    offset cannot stay in the product: it would grow with the number of keys
+//    summed into O);
 //  * V codes go into O^T += Vq^T P'^T unscaled, with each key's V scale folded
 //    into P: P' = p * s_v / s_max, where s_max is the largest V scale the warp
 //    has met so far (so P' stays in [0, 1], clear of fp16 subnormals).  When
@@ -251,16 +253,18 @@ __device__ __forceinline__ void mma_f16_16816(float* d, const uint32_t* a, uint3
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// S^T tile from int8 codes (A, 16 x 32) and int8 query parts (B, 32 x 8), int32 accumulate
+__device__ __forceinline__ void mma_s8_16832(int* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Two int8 codes (bytes 0 and 2 of u ^ 0x80808080 selected by sel) -> the
-// exact fp16 pair code + 1152 (the byte u = code + 128 under the exponent
-// pattern of 1024); the K path keeps the offset and removes it from S.
-__device__ __forceinline__ uint32_t codes_to_h2_off(uint32_t u_flipped, uint32_t sel) {
-  return __byte_perm(u_flipped, 0x64646464u, sel);                  // halves 0x64uu = 1024 + u
 }
 
 // Two int8 codes (bytes 0 and 2 of u ^ 0x80808080 selected by sel) -> exact fp16 pair.
@@ -282,47 +286,56 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int g = lane >> 2, c = lane & 3;
 
-  // ---- Q^T operand (fp16): head g, dims 32c + 4kc + {0, 1} (b0) and {2, 3} (b1)
-  uint32_t qb[8][2];
-  if (g < G) {
-    const __nv_bfloat16* qp =
-        reinterpret_cast<const __nv_bfloat16*>(a.q.ptr) + b * a.q.sb + (int64_t)(hk * G + g) * a.q.sh + 32 * c;
-    const int64_t qpos = a.positions ? a.positions[a.q_index] : a.q_index;
+  // ---- Q^T operand (int8 pair): head g, dims [32c, 32c + 32) of the rotated q,
+  // split as q = s_q (128 hi + lo) + e with hi in [-127, 127], lo in [-64, 64]
+  // and |e| <= s_q / 2, s_q = amax / (127 * 128) per head (15 bits, finer
+  // than the fp16 operand's 11).  Word w holds dims 32c + 4w .. 32c + 4w + 3.
+  uint32_t qhi[8], qlo[8];
+  float sqc[2];                                     // s_q of heads 2c, 2c + 1 (this lane's S columns)
+  {
+    float qf[32];
+    if (g < G) {
+      const __nv_bfloat16* qp =
+          reinterpret_cast<const __nv_bfloat16*>(a.q.ptr) + b * a.q.sb + (int64_t)(hk * G + g) * a.q.sh + 32 * c;
+      const int64_t qpos = a.positions ? a.positions[a.q_index] : a.q_index;
 #pragma unroll
-    for (int kc = 0; kc < 8; ++kc)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int d0 = 4 * kc + 2 * hf;
-        float2 x = bf2_to_f2(*reinterpret_cast<const uint32_t*>(qp + d0));
+      for (int i = 0; i < 16; ++i) {
+        float2 x = bf2_to_f2(*reinterpret_cast<const uint32_t*>(qp + 2 * i));
         if (a.rope_q) {
           float cs, sn;
-          rope_cos_sin(qpos, a.f.theta[16 * c + (d0 >> 1)], cs, sn);
+          rope_cos_sin(qpos, a.f.theta[16 * c + i], cs, sn);
           x = make_float2(x.x * cs - x.y * sn, x.x * sn + x.y * cs);
         }
-        qb[kc][hf] = f2_to_h2(x.x, x.y);
+        qf[2 * i] = x.x;
+        qf[2 * i + 1] = x.y;
       }
-  } else {
+    } else {
 #pragma unroll
-    for (int kc = 0; kc < 8; ++kc) qb[kc][0] = qb[kc][1] = 0u;
-  }
-
-  // K codes enter the S^T product as code + 1152, so S'^T = S^T + 1152 sum_d q_d
-  // per query head; qs[h] (h = 0, 1: heads 2c, 2c + 1, this lane's columns)
-  // is that sum over the same fp16 q values the MMA reads.
-  float qs[2];
-  {
-    float part = 0.f;
+      for (int i = 0; i < 32; ++i) qf[i] = 0.f;
+    }
+    float am = 0.f;
 #pragma unroll
-    for (int kc = 0; kc < 8; ++kc)
+    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(qf[i]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));     // lanes 4g .. 4g + 3 hold head g
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    const float inv = am > 0.f ? 16256.f / am : 0.f;
+    const float sq = am > 0.f ? am / 16256.f : 0.f;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&qb[kc][hf]);
-        part += __low2float(h) + __high2float(h);
+    for (int w = 0; w < 8; ++w) {
+      uint32_t ph = 0u, pl = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float y = qf[4 * w + e] * inv;
+        const float hi = rintf(y * (1.f / 128.f));
+        const int lo = __float2int_rn(y - 128.f * hi);
+        ph |= ((uint32_t)(int)hi & 0xffu) << (8 * e);
+        pl |= ((uint32_t)lo & 0xffu) << (8 * e);
       }
-    part += __shfl_xor_sync(0xffffffffu, part, 1);     // lanes 4g .. 4g + 3 hold head g
-    part += __shfl_xor_sync(0xffffffffu, part, 2);
-    qs[0] = __shfl_sync(0xffffffffu, part, 8 * c) * 1152.f;
-    qs[1] = __shfl_sync(0xffffffffu, part, 8 * c + 4) * 1152.f;
+      qhi[w] = ph;
+      qlo[w] = pl;
+    }
+    sqc[0] = __shfl_sync(0xffffffffu, sq, 8 * c);
+    sqc[1] = __shfl_sync(0xffffffffu, sq, 8 * c + 4);
   }
 
   // ---- this warp's key range, in kDqKeys-key tiles from k_lo
@@ -425,7 +438,7 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
     const float* sv_ = sk + kDqKeys;
     // S^T = Kq Q^T for the two 16-key halves u (keys 16u + g, 16u + g + 8 in
     // this lane's rows), dims [32c, 32c + 32) per lane: two independent chains
-    float sacc[2][4];
+    float sacc[2][4];                         // codes . (128 hi + lo) of the lane's (key, head) pairs
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       uint32_t kw[2][8];
@@ -437,15 +450,16 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
         kw[r][0] = u0.x; kw[r][1] = u0.y; kw[r][2] = u0.z; kw[r][3] = u0.w;
         kw[r][4] = u1.x; kw[r][5] = u1.y; kw[r][6] = u1.z; kw[r][7] = u1.w;
       }
+      // the codes are the A operand as they are: chunk kc is dims 32c + 8kc + [0, 8)
+      int shi[4] = {0, 0, 0, 0}, slo[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[u][e] = 0.f;
-#pragma unroll
-      for (int kc = 0; kc < 8; ++kc) {
-        const uint32_t fa = kw[0][kc] ^ 0x80808080u, fb = kw[1][kc] ^ 0x80808080u;
-        const uint32_t af[4] = {codes_to_h2_off(fa, 0x4140), codes_to_h2_off(fb, 0x4140),
-                                codes_to_h2_off(fa, 0x4342), codes_to_h2_off(fb, 0x4342)};
-        mma_f16_16816(sacc[u], af, qb[kc][0], qb[kc][1]);
+      for (int kc = 0; kc < 4; ++kc) {
+        const uint32_t af[4] = {kw[0][2 * kc], kw[1][2 * kc], kw[0][2 * kc + 1], kw[1][2 * kc + 1]};
+        mma_s8_16832(shi, af, qhi[2 * kc], qhi[2 * kc + 1]);
+        mma_s8_16832(slo, af, qlo[2 * kc], qlo[2 * kc + 1]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[u][e] = (float)(128 * shi[e] + slo[e]);   // exact: |S| < 2^29
     }
     // key scales of this lane's keys (u, r): 16u + g + 8r
     float skr[2][2], svr[2][2];
@@ -482,7 +496,7 @@ __global__ void __launch_bounds__(kDqWarps * 32) attn_decode_i8_kernel(const Dec
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = e >> 1;
-        sv[u][e] = vis[u][r] ? (sacc[u][e] - qs[e & 1]) * skr[u][r] * a.scale_log2 : -INFINITY;
+        sv[u][e] = vis[u][r] ? sacc[u][e] * (sqc[e & 1] * skr[u][r] * a.scale_log2) : -INFINITY;
       }
     float p[2][4], beta[2];
 #pragma unroll
