@@ -236,10 +236,12 @@ int rcx_kv_quantize_int8(rcx_tensor x, rcx_tensor codes, float* scale, void* str
  * rcx_attn_decode_int8_fwd -- rcx_attn_decode_fwd over an int8 KV cache made
  * by rcx_kv_quantize_int8: key j of KV head h stands for k_codes[j] *
  * k_scale[h, j] (and likewise V).  Same query, mask, GQA, temperature, LSE,
- * rope_flags and split-KV merge as rcx_attn_decode_fwd; the codes are
- * dequantised in the tile load and the contractions run in fp16 with fp32
- * accumulation, so |rotated q| and the dequantised V must stay below the fp16
- * range (65504).
+ * rope_flags and split-KV merge as rcx_attn_decode_fwd.  The logits come
+ * from int8 products of the stored K codes with each head's rotated query
+ * split into two int8 parts (15 bits of its largest element), times the
+ * scales; P V runs in fp16 with fp32 accumulation over the V codes with the V
+ * scales folded into P, so the result is the attention over the dequantised
+ * cache up to those roundings.
  *
  * q, o: [B, 1, Hq, 128] (q bf16; o bf16 or f32); k, v: [B, Nk, Hkv, 128]
  * RCX_I8, 16-byte aligned rows (base and strides multiples of 16 bytes);
