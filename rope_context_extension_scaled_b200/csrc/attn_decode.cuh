@@ -455,44 +455,67 @@ __global__ void __launch_bounds__(kDmWarps * 32) attn_decode_mma_kernel(const De
   }
 }
 
-// Merge the split partials of one (batch, head) row: thread per 4 dims.
+// Merge the key-range partials of each (batch, query head) row.
 template <typename Tout>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
+  // One CTA of 8 warps per (batch, query head) row: warp w merges key ranges
+  // w, w + 8, ... (lane c holds dims 4c .. 4c + 3), so the reads of all
+  // partials are spread over the CTA, and the 8 warp results merge in shared
+  // memory by the same LSE rule.
+  __shared__ float sm_m[8], sm_l[8];
+  __shared__ float4 sm_o[8][32];
   const int64_t rows = a.q.B * a.q.H;
-  const int64_t total = rows * 32;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = e / 32;
-    const int c = (int)(e % 32);
-    const int64_t b = row / a.q.H, h = row % a.q.H;
-    // max of the partial LSEs: lane c reads splits c, c + 32, ... and the row's
-    // 32 lanes (one warp) reduce, so the reads of all splits are in flight at once
+  const int warp = threadIdx.x / 32, c = threadIdx.x % 32;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     float mm = -INFINITY;
-    for (int s = c; s < a.splits; s += 32) mm = fmaxf(mm, a.part_lse[(int64_t)s * rows + row]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+    for (int s = warp; s < a.splits; s += 8) mm = fmaxf(mm, a.part_lse[(int64_t)s * rows + row]);
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lse = -INFINITY;
+    float wsum = 0.f;
     if (mm != -INFINITY) {
-      float wsum = 0.f;
-#pragma unroll 8
-      for (int s = 0; s < a.splits; ++s) {
+#pragma unroll 4
+      for (int s = warp; s < a.splits; s += 8) {
         const float ls = a.part_lse[(int64_t)s * rows + row];
         const float w = ls == -INFINITY ? 0.f : expf(ls - mm);
         const float4 x = *reinterpret_cast<const float4*>(a.part_o + ((int64_t)s * rows + row) * 128 + 4 * c);
         r.x += w * x.x; r.y += w * x.y; r.z += w * x.z; r.w += w * x.w;
         wsum += w;
       }
-      const float inv = 1.f / wsum;
-      r.x *= inv; r.y *= inv; r.z *= inv; r.w *= inv;
-      lse = mm + logf(wsum);
     }
-    Tout* op = reinterpret_cast<Tout*>(a.o.ptr) + b * a.o.sb + h * a.o.sh + 4 * c;
-    if constexpr (sizeof(Tout) == 2) {
-      *reinterpret_cast<uint2*>(op) = make_uint2(f2_to_bf2(r.x, r.y), f2_to_bf2(r.z, r.w));
-    } else {
-      *reinterpret_cast<float4*>(op) = r;
+    if (c == 0) {
+      sm_m[warp] = mm;
+      sm_l[warp] = wsum;
     }
-    if (c == 0 && a.lse) a.lse[b * a.lse_sb + h * a.lse_sh] = lse;
+    sm_o[warp][c] = r;
+    __syncthreads();
+    if (warp == 0) {
+      float mt = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) mt = fmaxf(mt, sm_m[w]);
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      float lse = -INFINITY;
+      if (mt != -INFINITY) {
+        float lt = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const float f = sm_m[w] == -INFINITY ? 0.f : expf(sm_m[w] - mt);
+          const float4 x = sm_o[w][c];
+          o.x += f * x.x; o.y += f * x.y; o.z += f * x.z; o.w += f * x.w;
+          lt += f * sm_l[w];
+        }
+        const float inv = 1.f / lt;
+        o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
+        lse = mt + logf(lt);
+      }
+      const int64_t b = row / a.q.H, h = row % a.q.H;
+      Tout* op = reinterpret_cast<Tout*>(a.o.ptr) + b * a.o.sb + h * a.o.sh + 4 * c;
+      if constexpr (sizeof(Tout) == 2) {
+        *reinterpret_cast<uint2*>(op) = make_uint2(f2_to_bf2(o.x, o.y), f2_to_bf2(o.z, o.w));
+      } else {
+        *reinterpret_cast<float4*>(op) = o;
+      }
+      if (c == 0 && a.lse) a.lse[b * a.lse_sb + h * a.lse_sh] = lse;
+    }
+    __syncthreads();
   }
 }
 

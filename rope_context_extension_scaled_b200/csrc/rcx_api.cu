@@ -412,8 +412,7 @@ int decode_impl(const rcx_tensor& q, const rcx_tensor& k, const rcx_tensor& v, c
     dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
     if ((st = decode_launch(a, (int)G, al(k, 16) && al(v, 16), grid, stream))) return st;
   }
-  const int64_t threads = B * Hq * 32;
-  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 8));
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(B * Hq, (int64_t)sm_count() * 8));   // a CTA per row
   return decode_combine_launch(a, o.dtype, grid2, stream);
 }
 
@@ -521,8 +520,7 @@ int decode_i8_impl(const rcx_tensor& q, const rcx_tensor& k, const float* k_scal
     dim3 grid((unsigned)p.splits, (unsigned)Hkv, (unsigned)B);
     if ((st = decode_i8_launch(a, (int)G, k_scale, v_scale, grid, stream))) return st;
   }
-  const int64_t threads = B * Hq * 32;
-  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>((threads + 255) / 256, (int64_t)sm_count() * 8));
+  const int grid2 = (int)std::max<int64_t>(1, std::min<int64_t>(B * Hq, (int64_t)sm_count() * 8));   // a CTA per row
   return decode_combine_launch(a, o.dtype, grid2, stream);
 }
 
