@@ -1,4 +1,4 @@
-"""Seeded random sweep of the attention paths against the float64 oracle.
+"""Seeded random sweeps of the attention and decode paths against the float64 oracle.
 
 Each case draws a shape (batch, tokens, query/KV heads with group sizes 1-8
 including odd ones), a RoPE schedule, a mask (causal, window, sinks), a ring
@@ -7,13 +7,15 @@ single-call kernel (tensor-core bf16 or SIMT fp32) or the multi-launch ring
 driver and compares every row with the oracle.  The draws are fixed by the
 case index, so a failure names a reproducible configuration."""
 
+import math
+
 import numpy as np
 import pytest
 import torch
 
 from rope_context_extension_scaled_b200 import _lib
 from rope_context_extension_scaled_b200.inputs import make_qkv
-from tests._parity import all_rows, assert_bf16, assert_f32, errors, gather_gpu, oracle_rows, schedule
+from tests._parity import all_rows, assert_bf16, assert_f32, errors, gather_gpu, np64, oracle_rows, schedule
 
 pytestmark = pytest.mark.gpu
 
@@ -83,3 +85,60 @@ def test_random_attention_configuration(case):
         assert err["lse_max"] <= 1e-2, err
     else:
         assert_bf16(err)
+
+
+def _draw_decode(case):
+    rng = np.random.default_rng(5000 + case)
+    B = int(rng.integers(1, 3))
+    Hkv = int(rng.choice([1, 2, 3, 4, 8]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    Nk = int(rng.integers(1, 6000))
+    window = int(rng.choice([0, 0, int(rng.integers(1, 3000))]))
+    n_sink = int(rng.integers(0, 6)) if window else 0
+    qoff = int(rng.choice([0, 0, int(rng.integers(1, 100))]))
+    scheme = SCHEMES[int(rng.integers(0, len(SCHEMES)))]
+    return dict(B=B, Hkv=Hkv, Hq=G * Hkv, Nk=Nk, window=window, n_sink=n_sink, qoff=qoff, scheme=scheme,
+                int8=bool(case % 2))
+
+
+@pytest.mark.parametrize("case", range(48))
+def test_random_decode_configuration(case):
+    # One query token per head against a cache of Nk keys, bf16 cache or its
+    # int8 codes (the oracle quantises with its own rule and attends over
+    # code * scale), every schedule, masks and a query past the cache.
+    from oracle import rcx_oracle as orc
+    c = _draw_decode(case)
+    B, Hq, Hkv, Nk = c["B"], c["Hq"], c["Hkv"], c["Nk"]
+    qf, _, _ = make_qkv(B, 1, Hq, Hkv, 128, torch.bfloat16, seed=6000 + case, device=DEV)
+    _, k, v = make_qkv(B, Nk, Hq, Hkv, 128, torch.bfloat16, seed=7000 + case, device=DEV)
+    inv, t, oinv, ot = schedule(c["scheme"], 5e5, 128, 4096, 65536)
+    krot = torch.empty_like(k)
+    _lib.rope_apply(None, k, inv, k_out=krot)                 # the cache holds rotated keys
+    q_index = Nk - 1 + c["qoff"]
+    pos = torch.arange(q_index + 1, dtype=torch.int64, device=DEV) if c["qoff"] else None
+    if c["int8"]:
+        kc, ks = _lib.kv_quantize_int8(krot)
+        vc, vs = _lib.kv_quantize_int8(v)
+        o, lse = _lib.attn_decode_int8_fwd(qf, kc, ks, vc, vs, window=c["window"], n_sink=c["n_sink"],
+                                           temperature=t, q_index=q_index, positions=pos, inv_freq=inv,
+                                           rope_flags=_lib.ROTATE_Q)
+    else:
+        o, lse = _lib.attn_decode_fwd(qf, krot, v, window=c["window"], n_sink=c["n_sink"], temperature=t,
+                                      q_index=q_index, positions=pos, inv_freq=inv, rope_flags=_lib.ROTATE_Q)
+    torch.cuda.synchronize()
+    for b in range(B):
+        q64 = orc.rope_rotate(np64(qf[b]), np.array([q_index]), oinv)          # [1, Hq, d]
+        if c["int8"]:
+            kcd, ksd = orc.quantize_kv_int8(krot[b].float().cpu().numpy())
+            vcd, vsd = orc.quantize_kv_int8(v[b].float().cpu().numpy())
+            kk, vv = orc.dequantize_kv_int8(kcd, ksd), orc.dequantize_kv_int8(vcd, vsd)
+        else:
+            kk, vv = np64(krot[b]), np64(v[b])
+        O, L = orc.attention(q64, kk, vv, 1.0 / (math.sqrt(128) * ot), window=c["window"], n_sink=c["n_sink"],
+                             q_index=np.array([q_index]), k_index=np.arange(Nk))
+        Og = {h: np64(o[b, 0, h, :])[None] for h in range(Hq)}
+        Lg = {h: np.array([float(lse[b, h, 0])]) for h in range(Hq)}
+        Or = {h: O[0][h][None] for h in range(Hq)}
+        Lr = {h: np.array([L[h, 0]]) for h in range(Hq)}
+        err = errors(Og, Lg, Or, Lr)
+        assert err["inf_ok"] and err["o_max"] <= 2e-2 and err["lse_max"] <= 1e-2, (c, err)
