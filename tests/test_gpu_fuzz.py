@@ -142,3 +142,59 @@ def test_random_decode_configuration(case):
         Lr = {h: np.array([L[h, 0]]) for h in range(Hq)}
         err = errors(Og, Lg, Or, Lr)
         assert err["inf_ok"] and err["o_max"] <= 2e-2 and err["lse_max"] <= 1e-2, (c, err)
+
+
+@pytest.mark.parametrize("case", range(32))
+def test_random_rope_apply_configuration(case):
+    # Q and K rotated in one call: random batch, tokens, heads, head widths,
+    # dtype, explicit positions, strided views (head slices of a packed tensor)
+    # and in-place or out-of-place outputs, against the oracle's rotation.
+    from oracle import rcx_oracle as orc
+    rng = np.random.default_rng(8000 + case)
+    f32 = bool(case % 2)
+    dt = torch.float32 if f32 else torch.bfloat16
+    per = 4 if f32 else 8                                # values per 16-byte piece
+    d = per * int(rng.integers(1, 256 // per + 1))
+    B, N = int(rng.integers(1, 4)), int(rng.integers(1, 400))
+    Hq, Hk = int(rng.integers(1, 9)), int(rng.integers(1, 5))
+    pad = int(rng.integers(0, 3))                        # extra heads in the packed tensor
+    g = torch.Generator(device="cpu")
+    g.manual_seed(9000 + case)
+    packed = torch.randn(B, N, Hq + Hk + pad, d, generator=g).to(dt).to(DEV)
+    q, k = packed[:, :, :Hq], packed[:, :, Hq:Hq + Hk]
+    pos = torch.randint(0, 1 << 20, (N,), generator=g, dtype=torch.int64).to(DEV) if rng.integers(0, 2) else None
+    inv, _, oinv, _ = schedule(SCHEMES[case % len(SCHEMES)], 1e4, d, 256, 4096)
+    q0, k0 = q.clone(), k.clone()
+    in_place = bool(rng.integers(0, 2))
+    qo, ko = (q, k) if in_place else (torch.empty_like(q0), torch.empty_like(k0))
+    _lib.rope_apply(q, k, inv, positions=pos, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    p_np = pos.cpu().numpy() if pos is not None else np.arange(N)
+    for x, y in ((q0, qo), (k0, ko)):
+        for b in range(B):
+            ref = orc.rope_rotate(np64(x[b]), p_np, oinv)
+            got = np64(y[b])
+            if f32:
+                assert np.abs(got - ref).max() < 1e-5, case
+            else:
+                assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5), case
+
+
+@pytest.mark.parametrize("case", range(24))
+def test_random_int8_quantise_configuration(case):
+    # Codes and scales bit-exact with the oracle for random batch, tokens,
+    # heads and magnitudes, packed or head-sliced caches (ties at half-codes
+    # are covered by the dedicated int8 tests).
+    from oracle import rcx_oracle as orc
+    rng = np.random.default_rng(9500 + case)
+    B, N, H = int(rng.integers(1, 3)), int(rng.integers(1, 3000)), int(rng.integers(1, 9))
+    pad = int(rng.integers(0, 2))
+    g = torch.Generator(device="cpu")
+    g.manual_seed(9600 + case)
+    base = torch.randn(B, N, H + pad, 128, generator=g) * float(rng.choice([0.01, 1.0, 30.0]))
+    x = base.to(torch.bfloat16).to(DEV)[:, :, :H]
+    codes, scale = _lib.kv_quantize_int8(x)
+    torch.cuda.synchronize()
+    c_ref, s_ref = orc.quantize_kv_int8(x.float().cpu().numpy())
+    assert np.array_equal(codes.cpu().numpy(), c_ref), case
+    assert np.array_equal(scale.permute(0, 2, 1).cpu().numpy(), s_ref), case
